@@ -1,0 +1,218 @@
+/*
+ * h3attn_oracle.c -- plain, slow, fp64 CPU oracle of the h3attn hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls
+ * this file; only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes (the method of the MiniMax-H3 denoiser's attention block):
+ *   - per-head Q/K RMSNorm followed by rotary position embedding, the fused
+ *     prologue the "H3 Runtime Current State" page lists as missing under
+ *     Owned Performance Kernels ("Fused Q/K RMSNorm, RoPE, and layout work"),
+ *     and that the "Buyer Questions Status" block-24 profile books as
+ *     "norm/RoPE" ahead of attention;
+ *   - non-causal softmax(Q K^T * scale) V over a packed video+audio token
+ *     sequence ("H3 Runtime Current State", Implemented And Validated: "H3
+ *     packed denoising"; "Open-H3-Regenerate-2K", Forward table: dense cuDNN
+ *     attention in standard_fwd), one sequence per cu_seqlens segment
+ *     ("Ragged Ulysses sequence parallelism").
+ *
+ * The pages print no formula for either step.  The readings taken here:
+ *   RMSNorm:  y = x / sqrt(mean(x^2) + eps) * gamma, over the head_dim values
+ *             of one (token, head) row; gamma shared by all heads.
+ *   RoPE:     adjacent pairs (x[2i], x[2i+1]) rotated by angle p * f_i:
+ *               y[2i]   = x[2i] cos a - x[2i+1] sin a
+ *               y[2i+1] = x[2i] sin a + x[2i+1] cos a
+ *             3D tokens: dims [0,st) use t, [st,st+sh) use h, the rest use w;
+ *             inside a section of width ds, pair i has f_i = theta^(-2i/ds).
+ *             1D tokens: one position over all dims, f_i = theta^(-2i/d).
+ *   Attention: s_j = scale * (q . k_j) over the keys of the query's sequence,
+ *             p_j = exp(s_j - max_j s_j), o = sum_j p_j v_j / sum_j p_j,
+ *             lse = max_j s_j + log(sum_j p_j).
+ *   Order:    RMSNorm, then RoPE, then one rounding to bfloat16 (nearest,
+ *             ties to even) -- the interface tensor attention consumes.
+ *
+ * Every loop below is the definition written out in double precision, in the
+ * order stated, with no blocking, fusion or reordering.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+int h3o_version(void) { return 1; }
+
+/* bfloat16 bit pattern -> double (exact). */
+double h3o_bf16_to_double(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* double -> nearest bfloat16 (8 significant bits, float32 exponent range),
+ * ties to even, rounded once from the double value. */
+uint16_t h3o_bf16_from_double(double x) {
+    if (isnan(x)) return (uint16_t)0x7FC0;
+    uint16_t sign = signbit(x) ? (uint16_t)0x8000 : (uint16_t)0;
+    double ax = fabs(x);
+    /* largest finite bf16 is 255 * 2^120; the midpoint to 2^128 is 511 * 2^119
+     * and ties go to the even neighbour, which is infinity. */
+    if (ax >= ldexp(511.0, 119)) return (uint16_t)(sign | 0x7F80);
+    double quantum;
+    if (ax < ldexp(1.0, -126)) {
+        quantum = ldexp(1.0, -133);            /* subnormal spacing */
+    } else {
+        int e;
+        frexp(ax, &e);                         /* ax in [2^(e-1), 2^e) */
+        quantum = ldexp(1.0, e - 1 - 7);       /* 7 stored mantissa bits */
+    }
+    double r = nearbyint(ax / quantum) * quantum; /* default mode: nearest-even */
+    float f = (float)r;                        /* exact: r is a bf16 value */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (uint16_t)(u >> 16));
+}
+
+void h3o_bf16_round_array(const double* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = h3o_bf16_from_double(x[i]);
+}
+
+/* Rotate the pair (row[i0], row[i0+1]) by angle a. */
+static void rotate_pair(double* row, int i0, double a) {
+    double c = cos(a), s = sin(a);
+    double x0 = row[i0], x1 = row[i0 + 1];
+    row[i0] = x0 * c - x1 * s;
+    row[i0 + 1] = x0 * s + x1 * c;
+}
+
+/* Rotary embedding of one row of length d for a token of the given kind. */
+static void rope_row(double* row, int d, int kind, const int32_t* p,
+                     int sec_t, int sec_h, int sec_w, double theta) {
+    if (kind == 1) {
+        int start[3] = {0, sec_t, sec_t + sec_h};
+        int width[3] = {sec_t, sec_h, sec_w};
+        for (int axis = 0; axis < 3; ++axis) {
+            for (int i = 0; i < width[axis] / 2; ++i) {
+                double f = pow(theta, -2.0 * (double)i / (double)width[axis]);
+                rotate_pair(row, start[axis] + 2 * i, (double)p[axis] * f);
+            }
+        }
+    } else if (kind == 2) {
+        for (int i = 0; i < d / 2; ++i) {
+            double f = pow(theta, -2.0 * (double)i / (double)d);
+            rotate_pair(row, 2 * i, (double)p[0] * f);
+        }
+    }
+}
+
+/*
+ * RMSNorm (if gamma != NULL) then RoPE (if pos != NULL and kind[n] != 0) of
+ * every (token, head) row of x.
+ *   x:      bf16 bits, row (n, h) starts at x + n*s_tok + h*s_head (elements).
+ *   gamma:  bf16 bits [d] or NULL.
+ *   pos:    int32 [n_tokens][3] or NULL;  kind: uint8 [n_tokens] (0, 1 = 3D, 2 = 1D).
+ *   y64:    double [n_tokens][n_heads][d] or NULL (unrounded result).
+ *   y16:    bf16 bits [n_tokens][n_heads][d] or NULL (result rounded once).
+ * Returns 0, or -1 on invalid arguments.
+ */
+int h3o_rmsnorm_rope(const uint16_t* x, int64_t n_tokens, int32_t n_heads, int32_t d,
+                     int64_t s_tok, int64_t s_head, const uint16_t* gamma, double eps,
+                     const int32_t* pos, const uint8_t* kind,
+                     int32_t sec_t, int32_t sec_h, int32_t sec_w, double theta,
+                     double* y64, uint16_t* y16) {
+    if (!x || n_tokens < 0 || n_heads <= 0 || d <= 0 || d > 1024 || (d & 1)) return -1;
+    if (pos && (!kind || sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t & 1) || (sec_h & 1) ||
+                (sec_w & 1) || sec_t + sec_h + sec_w != d))
+        return -1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < n_tokens; ++n) {
+        double row[1024];
+        for (int h = 0; h < n_heads; ++h) {
+            const uint16_t* src = x + n * s_tok + (int64_t)h * s_head;
+            for (int i = 0; i < d; ++i) row[i] = h3o_bf16_to_double(src[i]);
+            if (gamma) {
+                double ss = 0.0;
+                for (int i = 0; i < d; ++i) ss += row[i] * row[i];
+                double r = sqrt(ss / (double)d + eps);
+                for (int i = 0; i < d; ++i) row[i] = row[i] / r * h3o_bf16_to_double(gamma[i]);
+            }
+            if (pos && kind[n] != 0)
+                rope_row(row, d, kind[n], pos + 3 * n, sec_t, sec_h, sec_w, theta);
+            int64_t o = (n * n_heads + h) * (int64_t)d;
+            if (y64) for (int i = 0; i < d; ++i) y64[o + i] = row[i];
+            if (y16) for (int i = 0; i < d; ++i) y16[o + i] = h3o_bf16_from_double(row[i]);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Attention for selected query rows.
+ *   q, k, v:    bf16 bits, packed [total][n_heads][d].
+ *   cu_seqlens: int32 [nseq + 1], cu[0] = 0, non-decreasing, cu[nseq] = total.
+ *   rows:       int64 [nrows] global query token indices (NULL = all tokens).
+ *   o:          double [nrows][n_heads][d];  lse: double [nrows][n_heads] or NULL.
+ * A query attends to every key of its own sequence, none of any other.
+ * Returns 0, or -1 on invalid arguments.
+ */
+int h3o_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t total,
+                  int32_t n_heads, int32_t d, const int32_t* cu_seqlens, int32_t nseq,
+                  double scale, const int64_t* rows, int64_t nrows, double* o, double* lse) {
+    if (!q || !k || !v || !o || !cu_seqlens || total <= 0 || n_heads <= 0 || d <= 0 || d > 1024 ||
+        nseq <= 0)
+        return -1;
+    if (cu_seqlens[0] != 0 || cu_seqlens[nseq] != total) return -1;
+    for (int s = 0; s < nseq; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
+    if (!rows) nrows = total;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        if (t < 0 || t >= total) return -1;
+    }
+    double* kd = (double*)malloc(sizeof(double) * (size_t)total * (size_t)d);
+    double* vd = (double*)malloc(sizeof(double) * (size_t)total * (size_t)d);
+    if (!kd || !vd) { free(kd); free(vd); return -2; }
+    for (int h = 0; h < n_heads; ++h) {
+        /* this head's keys and values as doubles, [total][d] */
+        #pragma omp parallel for schedule(static)
+        for (int64_t j = 0; j < total; ++j) {
+            for (int i = 0; i < d; ++i) {
+                kd[j * d + i] = h3o_bf16_to_double(k[(j * n_heads + h) * (int64_t)d + i]);
+                vd[j * d + i] = h3o_bf16_to_double(v[(j * n_heads + h) * (int64_t)d + i]);
+            }
+        }
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t t = rows ? rows[r] : r;
+            int s = 0;
+            while (!(cu_seqlens[s] <= t && t < cu_seqlens[s + 1])) ++s;
+            int64_t j0 = cu_seqlens[s], j1 = cu_seqlens[s + 1];
+            double qd[1024];
+            for (int i = 0; i < d; ++i) qd[i] = h3o_bf16_to_double(q[(t * n_heads + h) * (int64_t)d + i]);
+            double* sc = (double*)malloc(sizeof(double) * (size_t)(j1 - j0));
+            double mx = -INFINITY;
+            for (int64_t j = j0; j < j1; ++j) {
+                double dot = 0.0;
+                for (int i = 0; i < d; ++i) dot += qd[i] * kd[j * d + i];
+                sc[j - j0] = scale * dot;
+                if (sc[j - j0] > mx) mx = sc[j - j0];
+            }
+            double acc[1024];
+            for (int i = 0; i < d; ++i) acc[i] = 0.0;
+            double den = 0.0;
+            for (int64_t j = j0; j < j1; ++j) {
+                double p = exp(sc[j - j0] - mx);
+                den += p;
+                for (int i = 0; i < d; ++i) acc[i] += p * vd[j * d + i];
+            }
+            double* out = o + (r * n_heads + h) * (int64_t)d;
+            for (int i = 0; i < d; ++i) out[i] = acc[i] / den;
+            if (lse) lse[r * n_heads + h] = mx + log(den);
+            free(sc);
+        }
+    }
+    free(kd);
+    free(vd);
+    return 0;
+}

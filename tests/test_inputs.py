@@ -1,0 +1,45 @@
+"""The seeded input generator: determinism, shapes and layout of the workloads."""
+import numpy as np
+
+from video_diffusion_transformer_h3attn_b200 import inputs
+
+
+def test_bf16_conversion_round_trip_and_ties():
+    x = np.array([1.0, -2.5, 1.00390625, 1.005859375, 3.0e38, 0.0], dtype=np.float32)
+    b = inputs.f32_to_bf16_bits(x)
+    # 1.00390625 is the midpoint of 1 and 1+2^-7: ties go to the even pattern (1.0)
+    assert list(b[:3]) == [0x3F80, 0xC020, 0x3F80]
+    # 1.005859375 = 1 + 3*2^-9 is above the midpoint -> rounds up to 1 + 2^-7
+    assert b[3] == 0x3F81
+    assert np.array_equal(inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(np.float32([0.75]))),
+                          np.float32([0.75]))
+
+
+def test_workloads_are_deterministic_and_shaped():
+    a = inputs.workload("tiny")
+    b = inputs.workload("tiny")
+    assert np.array_equal(a.q, b.q) and np.array_equal(a.v, b.v)
+    assert a.q.shape == (256, 2, 64) and a.pos is None and a.gamma_q is None
+    s = inputs.workload("small")
+    assert s.q.shape == (3072, 24, 128) and s.gamma_q.shape == (128,)
+    assert s.pos.shape == (3072, 3) and np.all(s.kind == inputs.KIND_3D)
+    # row-major (t, h, w): token 24*16 + 24 + 5 is (1, 1, 5)
+    assert tuple(s.pos[24 * 16 + 24 + 5]) == (1, 1, 5)
+    g = inputs.bf16_bits_to_f32(s.gamma_q)
+    assert g.min() >= 0.5 and g.max() <= 1.5
+
+
+def test_joint_and_ragged_layouts():
+    pos, kind = inputs.video_layout(16, 30, 54, 256)
+    assert len(pos) == 26176 and np.all(kind[:25920] == 1) and np.all(kind[25920:] == 2)
+    assert np.array_equal(pos[25920:, 0], np.arange(256))
+    pos, kind = inputs.ragged_layout([4096, 9000, 17001, 31234])
+    assert len(pos) == 61331 and pos[4096, 0] == 0 and pos[4095, 0] == 4095 and pos[-1, 0] == 31233
+
+
+def test_sample_rows_cover_boundaries():
+    cu = np.array([0, 300, 700])
+    rows = inputs.sample_rows(cu, 64, seed=1)
+    for r in (0, 299, 300, 699, 127, 128, 427, 428):
+        assert r in rows
+    assert rows.min() >= 0 and rows.max() < 700
