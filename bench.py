@@ -1,0 +1,398 @@
+"""Benchmark of the h3attn hot path on B200: one step = the Q/K RMSNorm + RoPE
+prologue followed by dense non-causal attention, on the 2K-refine workload
+(one clip of a 32 x 48 x 84 latent grid = 129,024 tokens, 24 heads of 128).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl h3attn|reference]
+
+Prints one JSON line (rank 0).  Metric: attention forward TFLOP/s counted as
+4 * N^2 * d * H per clip, whole job, max time over ranks.  With N GPUs every
+rank runs its own clip (weak scaling, no collective on the data path).
+
+--impl reference times the fp64 CPU oracle (the correctness reference of this
+project) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (4·N²·d·H) and % of B200 dense BF16 peak at N=129k"
+WORKLOAD = "2k"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workload_config(w, n_gpus):
+    return {
+        "workload": "2K refine clip: latent grid 32x48x84 = 129024 tokens, 24 heads x 128, "
+                    "Q/K RMSNorm (eps 1e-6) + 3D RoPE 32/48/48 (theta 1e4) + non-causal attention",
+        "global_batch": n_gpus,
+        "seq_len": int(w.total),
+        "heads": int(w.n_heads),
+        "head_dim": int(w.head_dim),
+        "parallelism": "replicas" if n_gpus == 1 else "dp%d" % n_gpus,
+        "l2": "inputs larger than L2 (Q, K, V 2.4 GB per clip)",
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# -----------------------------------------------------------------------------------------
+# clocks during the timed region
+# -----------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.samples = []
+        if self.proc is None:
+            return False
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "samples", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        pw = [float(s[3]) for s in self.samples if s[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for s in self.samples for n, v in zip(names, s[5:9]) if v.lower() == "active"})
+        loaded = [c for c, p in zip(sm, pw) if p > 0.5 * max(pw)] if pw else sm
+        return {"sm_mhz": statistics.median(loaded or sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples), "power_w_max": max(pw) if pw else None}
+
+
+# -----------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and --impl reference)
+# -----------------------------------------------------------------------------------------
+def _cores_used():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_setup(w, orc):
+    """K' of the whole clip (every query attends to all of it) -- done once."""
+    t0 = time.perf_counter()
+    _, k16 = orc.rmsnorm_rope(w.k, w.gamma_k, w.eps, w.pos, w.kind, w.sections, w.theta, want_f64=False)
+    return k16, time.perf_counter() - t0
+
+
+def oracle_sample_step(w, orc, k16, rows):
+    """Oracle prologue of the sampled query rows + attention of those rows over all keys."""
+    _, q16 = orc.rmsnorm_rope(w.q[rows], w.gamma_q, w.eps, w.pos[rows], w.kind[rows], w.sections,
+                              w.theta, want_f64=False)
+    # the oracle reads query rows by index: scatter the sampled rows into a full-size
+    # buffer (np.empty maps pages lazily, so only the sampled rows are touched)
+    qbuf = np.empty_like(w.q)
+    qbuf[rows] = q16
+    orc.attention(qbuf, k16, w.v, w.cu_seqlens, rows=rows)
+
+
+def cpu_baseline(w, rows_target_s=15.0):
+    import oracle
+    orc = oracle.get()
+    k16, t_k = oracle_sample_setup(w, orc)
+    rows = np.arange(4, dtype=np.int64) * 7919 % w.total
+    t0 = time.perf_counter()
+    oracle_sample_step(w, orc, k16, rows)
+    t_probe = time.perf_counter() - t0
+    n = int(max(4, min(w.total, len(rows) * rows_target_s / max(t_probe, 1e-3))))
+    rows = np.unique(np.linspace(0, w.total - 1, n).astype(np.int64))
+    t0 = time.perf_counter()
+    oracle_sample_step(w, orc, k16, rows)
+    t_rows = time.perf_counter() - t0
+    flops_rows = 4.0 * len(rows) * w.total * w.head_dim * w.n_heads
+    # whole-clip time: prologue of all Q and K rows (2x the K pass) + attention of every row
+    t_full = 2.0 * t_k + t_rows * w.total / len(rows)
+    return {
+        "value": w.attention_flops() / t_full / 1e12,
+        "unit": "TFLOP/s",
+        "cores": _cores_used(),
+        "kind": "oracle",
+        "sample": "%d of %d query rows x %d heads (full keys) + the K prologue of the whole clip; "
+                  "extrapolated linearly to the whole clip (rows are independent and equal cost)"
+                  % (len(rows), w.total, w.n_heads),
+        "sample_tflops": flops_rows / t_rows / 1e12,
+        "seconds": t_k + t_rows,
+    }
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from video_diffusion_transformer_h3attn_b200 import inputs
+    w = inputs.workload(WORKLOAD)
+    orc = oracle.get()
+    k16, _ = oracle_sample_setup(w, orc)
+    rng = np.random.default_rng(0)
+    n_rows = 8
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(w.total, n_rows, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle_sample_step(w, orc, k16, rows)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    step = statistics.mean(times)
+    flops = 4.0 * n_rows * w.total * w.head_dim * w.n_heads
+    value = flops / step / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores_used(), "kind": "oracle",
+                         "sample": "%d random query rows x %d heads per step (full keys; K prologue "
+                                   "done once before timing)" % (n_rows, w.n_heads)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -----------------------------------------------------------------------------------------
+# GPU arm
+# -----------------------------------------------------------------------------------------
+def source_hash():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "video_diffusion_transformer_h3attn_b200", "csrc"))):
+        with open(os.path.join(ROOT, "video_diffusion_transformer_h3attn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "attention_2k_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("source_hash") != source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import video_diffusion_transformer_h3attn_b200 as h3
+    from video_diffusion_transformer_h3attn_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        args.gpus = world
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    w = inputs.workload(WORKLOAD)
+    dev = torch.device("cuda", local)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    host = {
+        "q": bf16(w.q).pin_memory(), "k": bf16(w.k).pin_memory(), "v": bf16(w.v).pin_memory(),
+        "gq": bf16(w.gamma_q).pin_memory(), "gk": bf16(w.gamma_k).pin_memory(),
+        "pos": torch.from_numpy(w.pos).pin_memory(), "kind": torch.from_numpy(w.kind).pin_memory(),
+    }
+    d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    qp = torch.empty_like(d["q"])
+    kp = torch.empty_like(d["k"])
+    o = torch.empty_like(d["q"])
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    ev = {"pro": [], "att": []}
+
+    def step(record=False):
+        if record:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+        h3.prologue(d["q"], d["k"], qp, kp, d["gq"], d["gk"], w.eps, d["pos"], d["kind"], w.sections, w.theta)
+        if record:
+            e[1].record(stream)
+        h3.attention(qp, kp, d["v"], o)
+        if record:
+            e[2].record(stream)
+            ev["pro"].append((e[0], e[1]))
+            ev["att"].append((e[1], e[2]))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-resident timing ----
+    for _ in range(args.warmup):
+        step()
+    h3.device_status()
+    barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    h3.device_status()
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
+    att_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["att"])
+    pro_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["pro"])
+
+    # ---- end to end through the public API: host buffers in, result back to host ----
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o.numel() * o.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    flops = w.attention_flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    att_tflops = flops / (att_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    pro_bytes = 4.0 * w.total * w.n_heads * w.head_dim * 2 + 12.0 * w.total + w.total + 4 * w.head_dim
+    pro_gbs = pro_bytes / (pro_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": workload_config(w, world),
+        "pct_of_datasheet_2250": 100.0 * value / world / DATASHEET_BF16_TFLOPS,
+        "pct_of_measured_burst": 100.0 * value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+        "kernels_ms": {"prologue": pro_ms, "attention": att_ms},
+        "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": att_tflops / peak, "traffic": profiled_traffic(),
+                     "kernel": "attn_fwd_kernel<128,false>",
+                     "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long step)" % peak_src},
+        "roofline_prologue": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks.get("hbm_gbs"),
+                              "unit": "GB/s", "frac": pro_gbs / peaks.get("hbm_gbs", 6650.0),
+                              "peak_source": peak_src},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            line["cpu_baseline"] = cpu_baseline(w)
+        except Exception as exc:  # the baseline is reported, never required
+            line["cpu_baseline"] = {"value": None, "unit": "TFLOP/s", "cores": _cores_used(),
+                                    "kind": "oracle", "sample": "failed: %s" % exc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["h3attn", "reference"], default="h3attn")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "h3attn":
+        print("note: raising --warmup to 3", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,160 @@
+/*
+ * h3attn.h -- C ABI of the h3attn library: the attention hot path of a joint
+ * video/audio diffusion transformer block (MiniMax-H3), written for one NVIDIA
+ * B200 (sm_100a).
+ *
+ * The path: per-head Q/K RMSNorm + rotary position embedding (one prologue
+ * kernel), then non-causal softmax(Q K^T * scale) V over a packed token
+ * sequence (one attention kernel, dense or ragged).
+ *
+ * Sources of the operations (web pages about the H3 runtimes):
+ *   - "H3 Runtime Current State", Owned Performance Kernels: a fused Q/K
+ *     RMSNorm, RoPE and layout kernel is listed as missing; Implemented And
+ *     Validated: "H3 packed denoising" (video and audio tokens in one
+ *     sequence) and "Ragged Ulysses sequence parallelism" (ragged sequences).
+ *   - "Buyer Questions Status", block composition answer: in the profiled
+ *     DiT block, attention is the largest share of time and norm/RoPE feeds it;
+ *     strided-NHD Q/K/V (no copy of the QKV projection output) was a measured
+ *     saving.
+ *   - "Open-H3-Regenerate-2K", Forward table: the standard forward runs dense
+ *     attention on one B200.
+ *
+ * Conventions shared by every call
+ *   - Tensors are bfloat16, token-major "NHD": element (token n, head h, dim i)
+ *     lives at base + n*tok_stride + h*head_stride + i (strides in elements, the
+ *     last dimension contiguous).  Strided views of one fused QKV buffer are
+ *     accepted as they are: no copy is made.
+ *   - Every device pointer and every stride must be a multiple of 16 bytes
+ *     (strides: multiples of 8 elements); otherwise H3ATTN_ERR_MISALIGNED.
+ *   - The caller owns every buffer.  The library allocates and frees no device
+ *     memory; it holds one small static device word for error reporting.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) of the current device and runs asynchronously: no call
+ *     synchronises the device.  All argument checks happen on the host before
+ *     anything is enqueued; a failed check enqueues nothing.
+ *   - Device-side waits are bounded: a kernel that waits longer than about one
+ *     second on an internal barrier stops, records the failure in the device
+ *     error word and returns without writing its remaining outputs.
+ *     h3attn_device_status() reads that word.
+ *   - Calls with distinct output buffers may run concurrently.
+ */
+#ifndef H3ATTN_H
+#define H3ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    H3ATTN_OK = 0,
+    H3ATTN_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, bad section split, ... */
+    H3ATTN_ERR_UNSUPPORTED = 2,    /* head_dim not in {64, 128}, sizes beyond the kernel limits */
+    H3ATTN_ERR_MISALIGNED = 3,     /* pointer or stride not a multiple of 16 bytes */
+    H3ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (see h3attn_last_error) */
+    H3ATTN_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up on a bounded internal wait */
+} h3attn_status;
+
+/* Library version as 10000*major + 100*minor + patch. */
+int h3attn_version(void);
+
+/* Static text for a status code (never NULL). */
+const char* h3attn_status_string(int status);
+
+/* Human-readable detail of the last failure on the calling host thread, or "". */
+const char* h3attn_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads the device error word of the current
+ * device: H3ATTN_OK, or H3ATTN_ERR_DEVICE_TIMEOUT if any kernel of this
+ * library gave up on a bounded wait since the word was last cleared, or
+ * H3ATTN_ERR_CUDA if the stream reports an error.  clear != 0 resets the word.
+ */
+int h3attn_device_status(void* stream, int clear);
+
+/*
+ * h3attn_prologue -- per-head RMSNorm of Q and K followed by rotary position
+ * embedding, rounded once to bfloat16.
+ *
+ * For every token n < n_tokens and head h < n_heads, on the row x of length
+ * head_dim (Q and K alike, each with its own gamma):
+ *   RMSNorm (skipped when that tensor's gamma is NULL):
+ *       x_i <- x_i / sqrt(mean_j(x_j^2) + eps) * gamma_i
+ *   RoPE (skipped when pos is NULL, or for tokens with kind[n] == 0):
+ *       pair (x_{2i}, x_{2i+1}) rotated by angle a_i:
+ *         y_{2i} = x_{2i} cos a_i - x_{2i+1} sin a_i,
+ *         y_{2i+1} = x_{2i} sin a_i + x_{2i+1} cos a_i
+ *       kind 1 (video, 3D): dims [0, sec_t) use pos[n][0] (t), [sec_t, sec_t+sec_h)
+ *         use pos[n][1] (h), the rest use pos[n][2] (w); inside a section of
+ *         width ds the i-th pair has a_i = p * theta^(-2i/ds).
+ *       kind 2 (audio or ragged, 1D): a_i = pos[n][0] * theta^(-2i/head_dim).
+ *   The result is rounded to the nearest bfloat16 once.
+ *
+ * q_in, k_in:   bf16 input rows, strides in_tok_stride / in_head_stride.
+ * q_out, k_out: bf16 output rows, strides out_tok_stride / out_head_stride.
+ *               In place is allowed (q_out == q_in with equal strides); other
+ *               overlaps between inputs and outputs are not.
+ * gamma_q, gamma_k: bf16 [head_dim] or NULL.     eps: added inside the sqrt.
+ * pos:   device int32 [n_tokens][3] or NULL;  kind: device uint8 [n_tokens]
+ *        (required when pos is given; values other than 0, 1, 2 act as 0).
+ * sec_t + sec_h + sec_w must equal head_dim, each even (checked only when pos
+ * is given).  head_dim: 64 or 128.  n_tokens == 0 is a no-op.
+ * Arithmetic: sum of squares and scaling in fp32; the rotation in fp64 from
+ * fp64 angles, so every output is within one bf16 ulp of the exactly rounded
+ * result.
+ */
+h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                              int64_t n_tokens, int32_t n_heads, int32_t head_dim,
+                              int64_t in_tok_stride, int64_t in_head_stride,
+                              int64_t out_tok_stride, int64_t out_head_stride,
+                              const void* gamma_q, const void* gamma_k, double eps,
+                              const int32_t* pos, const uint8_t* kind,
+                              int32_t sec_t, int32_t sec_h, int32_t sec_w, double theta,
+                              void* stream);
+
+/*
+ * h3attn_fwd -- dense non-causal attention over `batch` sequences of equal
+ * length seqlen:  O = softmax(Q K^T * scale) V  per (sequence, head).
+ *
+ * q, k, v, o: bf16 [batch][seqlen][n_heads][head_dim]; each has strides
+ *   {batch, token, head} in elements (x_strides[0..2]), last dim contiguous.
+ * softmax_scale <= 0 selects 1/sqrt(head_dim).
+ * lse: NULL, or fp32 [batch][n_heads][seqlen] receiving the natural-log
+ *   log-sum-exp of each row's scaled scores.
+ * head_dim: 64 or 128; seqlen >= 1 (any value, no multiple of 128 needed);
+ * n_heads >= 1; batch >= 1.  Rows of `o` outside the tensor are never written.
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation; softmax in
+ * fp32 with exp2; P rounded to bf16 for the PV product; O rounded to bf16.
+ */
+h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o,
+                         int32_t batch, int64_t seqlen, int32_t n_heads, int32_t head_dim,
+                         const int64_t q_strides[3], const int64_t k_strides[3],
+                         const int64_t v_strides[3], const int64_t o_strides[3],
+                         float softmax_scale, float* lse, void* stream);
+
+/*
+ * h3attn_fwd_varlen -- the same attention over nseq ragged sequences packed
+ * along the token dimension: sequence s owns tokens [cu_seqlens[s],
+ * cu_seqlens[s+1]) and attends only to its own keys.
+ *
+ * q, k, v, o: bf16 [total_tokens][n_heads][head_dim], strides {token, head}.
+ * cu_seqlens: DEVICE int32 [nseq + 1], cu_seqlens[0] = 0, non-decreasing,
+ *   cu_seqlens[nseq] = total_tokens (not checked on the host: it is device
+ *   memory; empty sequences are allowed and produce nothing).
+ * max_seqlen: host value >= every sequence length (sizes the launch).
+ * lse: NULL, or fp32 [n_heads][total_tokens].
+ * nseq <= 65535.  Other rules as h3attn_fwd.
+ */
+h3attn_status h3attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                const int32_t* cu_seqlens, int32_t nseq, int64_t total_tokens,
+                                int32_t max_seqlen, int32_t n_heads, int32_t head_dim,
+                                const int64_t q_strides[2], const int64_t k_strides[2],
+                                const int64_t v_strides[2], const int64_t o_strides[2],
+                                float softmax_scale, float* lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3ATTN_H */

@@ -1,0 +1,138 @@
+"""Parity of the CUDA attention kernels (dense and ragged) with the fp64 oracle.
+
+Both sides read the same bf16 Q', K' (the oracle's prologue output, rounded
+once) and V.  Small workloads are compared on every output; the large ones,
+launched at full size exactly as the benchmark launches them, on sampled query
+rows (every sequence's first and last rows, both sides of 128-row tile
+boundaries, and random rows), for which the oracle's result is exact."""
+import numpy as np
+import pytest
+
+import oracle
+from h3_testlib import check_attention, from_cuda_bf16, to_cuda_bf16, bf16_bits_to_f64
+from video_diffusion_transformer_h3attn_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h3():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import video_diffusion_transformer_h3attn_b200 as mod
+    return mod
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.get()
+
+
+_QK_CACHE = {}
+
+
+def _qk(orc, w):
+    """Q', K' (bf16 bits) of a workload from the oracle's prologue."""
+    if w.name not in _QK_CACHE:
+        (_, q16), (_, k16) = orc.prologue_workload(w)
+        _QK_CACHE[w.name] = (q16, k16)
+    return _QK_CACHE[w.name]
+
+
+def _gpu_dense(h3, q, k, v, lse=True):
+    import torch
+    qt, kt, vt = to_cuda_bf16(q), to_cuda_bf16(k), to_cuda_bf16(v)
+    o, l = h3.attention(qt, kt, vt, return_lse=True)
+    h3.device_status()
+    return from_cuda_bf16(o), l.cpu().numpy()
+
+
+def _gpu_varlen(h3, q, k, v, cu):
+    import torch
+    qt, kt, vt = to_cuda_bf16(q), to_cuda_bf16(k), to_cuda_bf16(v)
+    cut = torch.from_numpy(np.asarray(cu, dtype=np.int32)).cuda()
+    maxlen = int(np.max(np.diff(cu))) if len(cu) > 1 else 1
+    o, l = h3.attention_varlen(qt, kt, vt, cut, max(1, maxlen), return_lse=True)
+    h3.device_status()
+    return from_cuda_bf16(o), l.cpu().numpy()
+
+
+def test_tiny_full(h3, orc):
+    w = inputs.workload("tiny")
+    o, lse = _gpu_dense(h3, w.q, w.k, w.v)
+    ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "tiny", lse.T, rl)
+
+
+def test_small_full(h3, orc):
+    w = inputs.workload("small")
+    q, k = _qk(orc, w)
+    o, lse = _gpu_dense(h3, q, k, w.v)
+    ro, rl = orc.attention(q, k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "small", lse.T, rl)
+
+
+@pytest.mark.parametrize("name,n_rows", [("joint", 384), ("2k", 160)])
+def test_large_sampled(h3, orc, name, n_rows):
+    w = inputs.workload(name)
+    q, k = _qk(orc, w)
+    o, lse = _gpu_dense(h3, q, k, w.v)
+    rows = inputs.sample_rows(w.cu_seqlens, n_rows, seed=w.seed + 1000)
+    ro, rl = orc.attention(q, k, w.v, w.cu_seqlens, rows=rows)
+    check_attention(bf16_bits_to_f64(o[rows]), ro, name, lse.T[rows], rl)
+
+
+def test_ragged_sampled(h3, orc):
+    w = inputs.workload("ragged")
+    q, k = _qk(orc, w)
+    o, lse = _gpu_varlen(h3, q, k, w.v, w.cu_seqlens)
+    rows = inputs.sample_rows(w.cu_seqlens, 384, seed=w.seed + 1000)
+    ro, rl = orc.attention(q, k, w.v, w.cu_seqlens, rows=rows)
+    check_attention(bf16_bits_to_f64(o[rows]), ro, "ragged", lse.T[rows], rl)
+
+
+@pytest.mark.parametrize("n", [1, 2, 127, 128, 129, 255, 256, 257, 383, 640])
+@pytest.mark.parametrize("d", [64, 128])
+def test_edge_lengths(h3, orc, n, d):
+    w = inputs.random_case([n], 3, d, seed=500 + n + d)
+    o, lse = _gpu_dense(h3, w.q, w.k, w.v)
+    ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "n=%d d=%d" % (n, d), lse.T, rl)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_edges(h3, orc, d):
+    lens = [1, 130, 0, 255, 4, 513, 128]
+    w = inputs.random_case(lens, 2, d, seed=900 + d, q_scale=3.0)
+    o, lse = _gpu_varlen(h3, w.q, w.k, w.v, w.cu_seqlens)
+    ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "ragged edges d=%d" % d, lse.T, rl)
+
+
+def test_batched_strided_views(h3, orc):
+    """B = 2 sequences read through strided views of one fused [B, N, 3, H, d] QKV buffer."""
+    import torch
+    B, N, H, d = 2, 300, 4, 128
+    w = inputs.random_case([N] * B, H, d, seed=31)
+    buf = torch.zeros((B, N, 3, H, d), dtype=torch.bfloat16, device="cuda")
+    for i, a in enumerate((w.q, w.k, w.v)):
+        buf[:, :, i] = to_cuda_bf16(a).view(B, N, H, d)
+    o = h3.attention(buf[:, :, 0], buf[:, :, 1], buf[:, :, 2])
+    h3.device_status()
+    got = bf16_bits_to_f64(from_cuda_bf16(o)).reshape(B * N, H, d)
+    ro, _ = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(got, ro, "batched strided")
+
+
+def test_special_cases(h3, orc):
+    """Q = 0 gives the mean of V; constant V rows give that row (to rounding)."""
+    w = inputs.random_case([700], 2, 128, seed=41)
+    zero = np.zeros_like(w.q)
+    o, _ = _gpu_dense(h3, zero, w.k, w.v)
+    mean = bf16_bits_to_f64(w.v).mean(axis=0)
+    check_attention(bf16_bits_to_f64(o), np.broadcast_to(mean, o.shape), "Q=0")
+    vc = np.broadcast_to(w.v[5], w.v.shape).copy()
+    o, _ = _gpu_dense(h3, w.q, w.k, vc)
+    check_attention(bf16_bits_to_f64(o), bf16_bits_to_f64(vc), "constant V")
+    assert np.mean(o == vc) > 0.99, "constant V rows should come back (almost always) exactly"

@@ -1,0 +1,109 @@
+"""The C ABI without a GPU: the library loads, exports what include/h3attn.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+
+import pytest
+
+import video_diffusion_transformer_h3attn_b200 as h3
+from video_diffusion_transformer_h3attn_b200 import _build
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced on the host
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return h3.library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = h3.declared_symbols()
+    assert set(names) >= {"h3attn_prologue", "h3attn_fwd", "h3attn_fwd_varlen", "h3attn_version",
+                          "h3attn_status_string", "h3attn_last_error", "h3attn_device_status"}
+    for n in names:
+        assert hasattr(lib, n), "library does not export %s" % n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.h3attn_version() >= 10000
+    for code in range(6):
+        assert lib.h3attn_status_string(code)
+    assert lib.h3attn_status_string(99) == b"unknown status"
+
+
+S3 = ctypes.c_int64 * 3
+S2 = ctypes.c_int64 * 2
+
+
+def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, N=256, H=2, d=64, strides=(256 * 128, 128, 64),
+        scale=0.0, lse=None):
+    s = S3(*strides)
+    return lib.h3attn_fwd(q, k, v, o, B, N, H, d, s, s, s, s, scale, lse, None)
+
+
+def test_fwd_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == INVALID
+    assert fwd(lib, d=96) == UNSUPPORTED
+    assert fwd(lib, d=256) == UNSUPPORTED
+    assert b"head_dim" in lib.h3attn_last_error()
+    assert fwd(lib, H=0) == INVALID
+    assert fwd(lib, N=0) == INVALID
+    assert fwd(lib, B=0) == INVALID
+    assert fwd(lib, q=FAKE + 2) == MISALIGNED
+    assert fwd(lib, strides=(256 * 128, 130, 64)) == MISALIGNED
+    assert fwd(lib, strides=(256 * 128, -128, 64)) == INVALID
+    assert fwd(lib, scale=float("inf")) == INVALID
+    assert fwd(lib, lse=FAKE + 2) == MISALIGNED
+    assert b"lse" in lib.h3attn_last_error()
+
+
+def varlen(lib, cu=FAKE, nseq=2, total=300, max_seqlen=200, H=2, d=128, strides=(256, 128)):
+    s = S2(*strides)
+    return lib.h3attn_fwd_varlen(FAKE, FAKE, FAKE, FAKE, cu, nseq, total, max_seqlen, H, d, s, s, s, s,
+                                 0.0, None, None)
+
+
+def test_varlen_rejects_bad_arguments(lib):
+    assert varlen(lib, cu=None) == INVALID
+    assert varlen(lib, nseq=0) == INVALID
+    assert varlen(lib, total=0) == INVALID
+    assert varlen(lib, max_seqlen=0) == INVALID
+    assert varlen(lib, max_seqlen=301) == INVALID
+    assert varlen(lib, d=80) == UNSUPPORTED
+    assert varlen(lib, strides=(257, 128)) == MISALIGNED
+
+
+def prologue(lib, n=10, H=2, d=128, gq=FAKE, pos=FAKE, kind=FAKE, sec=(32, 48, 48), eps=1e-6,
+             theta=1e4, strides=(256, 128, 256, 128), q=FAKE):
+    return lib.h3attn_prologue(q, FAKE, FAKE, FAKE, n, H, d, *strides, gq, FAKE, eps, pos, kind,
+                               sec[0], sec[1], sec[2], theta, None)
+
+
+def test_prologue_rejects_bad_arguments(lib):
+    assert prologue(lib, q=None) == INVALID
+    assert prologue(lib, d=96) == UNSUPPORTED
+    assert prologue(lib, n=-1) == INVALID
+    assert prologue(lib, H=0) == INVALID
+    assert prologue(lib, sec=(32, 48, 50)) == INVALID      # does not sum to d
+    assert prologue(lib, sec=(31, 49, 48)) == INVALID      # odd sections
+    assert prologue(lib, kind=None) == INVALID              # pos without kind
+    assert prologue(lib, theta=0.0) == INVALID
+    assert prologue(lib, eps=-1.0) == INVALID
+    assert prologue(lib, gq=FAKE + 8) == MISALIGNED
+    assert prologue(lib, strides=(256, 128, 252, 128)) == MISALIGNED
+
+
+def test_prologue_empty_is_a_no_op(lib):
+    # zero tokens: validated, nothing enqueued, no device needed
+    assert prologue(lib, n=0) == OK
+    assert prologue(lib, n=0, pos=None, kind=None) == OK
+
+
+def test_python_binding_refuses_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        h3.attention(x, x, x)
+    with pytest.raises(TypeError):
+        h3.prologue(x, x)

@@ -1,0 +1,125 @@
+"""Parity of the CUDA prologue (RMSNorm + RoPE) with the fp64 oracle: every
+output element within one bf16 ulp of the oracle's correctly rounded value."""
+import numpy as np
+import pytest
+
+import oracle
+from h3_testlib import check_prologue, from_cuda_bf16, to_cuda_bf16
+from video_diffusion_transformer_h3attn_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h3():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import video_diffusion_transformer_h3attn_b200 as mod
+    return mod
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.get()
+
+
+def _cuda(a, dtype=None):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.cuda() if dtype is None else t.to(dtype).cuda()
+
+
+def _run(h3, w, tokens=None, fused=False, in_place=False):
+    """GPU prologue of a workload (optionally a token subset); returns (q', k') bits."""
+    import torch
+    q, k = w.q, w.k
+    pos, kind = w.pos, w.kind
+    if tokens is not None:
+        q, k = q[tokens], k[tokens]
+        pos = None if pos is None else pos[tokens]
+        kind = None if kind is None else kind[tokens]
+    n, H, d = q.shape
+    if fused:
+        # one [n, 3, H, d] buffer, Q and K as strided views (the QKV projection layout)
+        buf = torch.zeros((n, 3, H, d), dtype=torch.bfloat16, device="cuda")
+        buf[:, 0] = to_cuda_bf16(q)
+        buf[:, 1] = to_cuda_bf16(k)
+        qt, kt = buf[:, 0], buf[:, 1]
+    else:
+        qt, kt = to_cuda_bf16(q), to_cuda_bf16(k)
+    gq = None if w.gamma_q is None else to_cuda_bf16(w.gamma_q)
+    gk = None if w.gamma_k is None else to_cuda_bf16(w.gamma_k)
+    pt = None if pos is None else _cuda(pos)
+    kd = None if kind is None else _cuda(kind)
+    outs = (qt, kt) if in_place else (None, None)
+    qo, ko = h3.prologue(qt, kt, outs[0], outs[1], gq, gk, w.eps, pt, kd, w.sections, w.theta)
+    h3.device_status()
+    return from_cuda_bf16(qo), from_cuda_bf16(ko)
+
+
+def _ref(orc, w, tokens=None):
+    q, k, pos, kind = w.q, w.k, w.pos, w.kind
+    if tokens is not None:
+        q, k = q[tokens], k[tokens]
+        pos = None if pos is None else pos[tokens]
+        kind = None if kind is None else kind[tokens]
+    _, q16 = orc.rmsnorm_rope(q, w.gamma_q, w.eps, pos, kind, w.sections, w.theta, want_f64=False)
+    _, k16 = orc.rmsnorm_rope(k, w.gamma_k, w.eps, pos, kind, w.sections, w.theta, want_f64=False)
+    return q16, k16
+
+
+@pytest.mark.parametrize("name", ["small", "joint", "ragged"])
+def test_prologue_workloads(h3, orc, name):
+    w = inputs.workload(name)
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, name + " q")
+    check_prologue(gk, rk, name + " k")
+
+
+def test_prologue_2k_sampled_tokens(h3, orc):
+    w = inputs.workload("2k")
+    rng = np.random.default_rng(4)
+    tokens = np.unique(np.concatenate([[0, 1, 127, 128, len(w.q) - 1], rng.integers(0, len(w.q), 4096)]))
+    gq, gk = _run(h3, w)  # the full-size launch, as the benchmark runs it
+    rq, rk = _ref(orc, w, tokens)
+    check_prologue(gq[tokens], rq, "2k q")
+    check_prologue(gk[tokens], rk, "2k k")
+
+
+def test_prologue_fused_qkv_in_place(h3, orc):
+    w = inputs.workload("small")
+    gq, gk = _run(h3, w, fused=True, in_place=True)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "fused in-place q")
+    check_prologue(gk, rk, "fused in-place k")
+
+
+def test_prologue_d64_odd_heads_mixed_kinds(h3, orc):
+    # d = 64 packs two heads per warp pass: an odd head count exercises the tail;
+    # kinds 0/1/2 and a gamma on Q only exercise every branch
+    n, H, d = 333, 3, 64
+    w = inputs.make_workload("d64", [n], H, d, seed=77, norm=True, sections=(16, 24, 24))
+    rng = np.random.default_rng(78)
+    w.pos = np.stack([rng.integers(0, 40, n), rng.integers(0, 50, n), rng.integers(0, 90, n)], 1).astype(np.int32)
+    w.kind = rng.integers(0, 3, n).astype(np.uint8)
+    w.gamma_k = None
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "d64 q")
+    check_prologue(gk, rk, "d64 k")
+
+
+def test_prologue_norm_only_and_single_token(h3, orc):
+    w = inputs.make_workload("one", [1], 24, 128, seed=79, norm=True)
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "single token q")
+    check_prologue(gk, rk, "single token k")
+
+
+def test_prologue_identity_without_norm_or_rope(h3):
+    w = inputs.make_workload("copy", [100], 4, 128, seed=80, norm=False)
+    gq, gk = _run(h3, w)
+    assert np.array_equal(gq, w.q) and np.array_equal(gk, w.k)

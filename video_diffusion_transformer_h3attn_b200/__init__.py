@@ -1,0 +1,217 @@
+"""h3attn -- B200 (sm_100a) attention hot path of a joint video/audio DiT block.
+
+Python binding of the C ABI in include/h3attn.h.  It only marshals arguments
+(data pointers, strides, the current CUDA stream) into the library; every step
+of the computation runs in the library's CUDA kernels.  There is no CPU
+fallback: without the built library, or with tensors that are not CUDA bf16,
+the calls raise.
+
+    prologue(q, k, ...)                 per-head RMSNorm + RoPE of Q and K
+    attention(q, k, v, ...)             dense non-causal softmax(QK^T*scale)V
+    attention_varlen(q, k, v, cu, ...)  the same over ragged packed sequences
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional, Sequence, Tuple
+
+from . import _build
+
+__all__ = ["prologue", "attention", "attention_varlen", "device_status", "library", "H3AttnError",
+           "KIND_NONE", "KIND_3D", "KIND_1D", "declared_symbols"]
+
+KIND_NONE, KIND_3D, KIND_1D = 0, 1, 2
+
+LIBRARY_PATH = _build.LIBRARY
+HEADER_PATH = os.path.join(_build.INCLUDE, "h3attn.h")
+
+
+class H3AttnError(RuntimeError):
+    """A call into the h3attn library returned an error status."""
+
+    def __init__(self, call: str, status: int, detail: str):
+        self.status = status
+        super().__init__("%s failed: %s (%d): %s" % (call, _status_string(status), status, detail))
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_I64_3 = ctypes.c_int64 * 3
+_I64_2 = ctypes.c_int64 * 2
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libh3attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIBRARY_PATH):
+            raise RuntimeError("libh3attn.so is not built (%s); run __graft_entry__.build() or "
+                               "python -m video_diffusion_transformer_h3attn_b200._build" % LIBRARY_PATH)
+        lib = ctypes.CDLL(LIBRARY_PATH)
+        lib.h3attn_version.restype = ctypes.c_int
+        lib.h3attn_status_string.restype = ctypes.c_char_p
+        lib.h3attn_status_string.argtypes = [ctypes.c_int]
+        lib.h3attn_last_error.restype = ctypes.c_char_p
+        lib.h3attn_device_status.restype = ctypes.c_int
+        lib.h3attn_device_status.argtypes = [_P, ctypes.c_int]
+        lib.h3attn_prologue.restype = ctypes.c_int
+        lib.h3attn_prologue.argtypes = [_P, _P, _P, _P, _I64, _I32, _I32, _I64, _I64, _I64, _I64,
+                                        _P, _P, ctypes.c_double, _P, _P, _I32, _I32, _I32,
+                                        ctypes.c_double, _P]
+        lib.h3attn_fwd.restype = ctypes.c_int
+        lib.h3attn_fwd.argtypes = [_P, _P, _P, _P, _I32, _I64, _I32, _I32, _I64_3, _I64_3, _I64_3,
+                                   _I64_3, ctypes.c_float, _P, _P]
+        lib.h3attn_fwd_varlen.restype = ctypes.c_int
+        lib.h3attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I64_2,
+                                          _I64_2, _I64_2, _I64_2, ctypes.c_float, _P, _P]
+        _lib = lib
+    return _lib
+
+
+def declared_symbols() -> list:
+    """Names of the functions include/h3attn.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(h3attn_[a-z_]+)\s*\(", text)))
+
+
+def _status_string(status: int) -> str:
+    try:
+        return library().h3attn_status_string(status).decode()
+    except Exception:  # pragma: no cover - only when the library is missing
+        return "status"
+
+
+def _check(call: str, status: int) -> None:
+    if status != 0:
+        raise H3AttnError(call, status, library().h3attn_last_error().decode())
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _require_bf16_cuda(name: str, t) -> None:
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError("%s must be a CUDA bfloat16 tensor" % name)
+    if t.stride(-1) != 1:
+        raise ValueError("%s: the last dimension must be contiguous" % name)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def device_status(stream=None, clear: bool = True) -> None:
+    """Synchronise `stream` and raise if a kernel recorded a device-side timeout."""
+    _check("h3attn_device_status", library().h3attn_device_status(_stream_handle(stream), int(clear)))
+
+
+def prologue(q, k, q_out=None, k_out=None, gamma_q=None, gamma_k=None, eps: float = 1e-6,
+             pos=None, kind=None, sections: Sequence[int] = (32, 48, 48), theta: float = 10000.0,
+             stream=None) -> Tuple[object, object]:
+    """RMSNorm (when gamma is given) then RoPE (when pos is given) of q and k.
+
+    q, k: bf16 CUDA [n_tokens, n_heads, head_dim] views with equal strides (e.g. two
+    slices of one fused QKV buffer).  q_out/k_out default to new contiguous tensors;
+    pass q_out=q, k_out=k for in-place.  pos: int32 [n_tokens, 3]; kind: uint8 [n_tokens].
+    """
+    torch = _torch()
+    _require_bf16_cuda("q", q)
+    _require_bf16_cuda("k", k)
+    if q.dim() != 3 or q.shape != k.shape or q.stride() != k.stride():
+        raise ValueError("q and k must be [n_tokens, n_heads, head_dim] with equal shapes and strides")
+    if q_out is None:
+        q_out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    if k_out is None:
+        k_out = torch.empty(k.shape, dtype=k.dtype, device=k.device)
+    _require_bf16_cuda("q_out", q_out)
+    _require_bf16_cuda("k_out", k_out)
+    if q_out.shape != q.shape or q_out.stride() != k_out.stride():
+        raise ValueError("q_out and k_out must match q's shape and share strides")
+    for name, g in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        if g is not None:
+            _require_bf16_cuda(name, g)
+    if pos is not None:
+        if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous():
+            raise TypeError("pos must be a contiguous CUDA int32 tensor [n_tokens, 3]")
+        if kind is None or kind.dtype != torch.uint8 or not kind.is_cuda or not kind.is_contiguous():
+            raise TypeError("kind must be a contiguous CUDA uint8 tensor [n_tokens]")
+    n, h, d = q.shape
+    st, sh, sw = sections
+    _check("h3attn_prologue", library().h3attn_prologue(
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), n, h, d, q.stride(0), q.stride(1),
+        q_out.stride(0), q_out.stride(1), _ptr(gamma_q), _ptr(gamma_k), float(eps), _ptr(pos),
+        _ptr(kind), st, sh, sw, float(theta), _stream_handle(stream)))
+    return q_out, k_out
+
+
+def attention(q, k, v, o=None, softmax_scale: Optional[float] = None, return_lse: bool = False,
+              stream=None):
+    """softmax(q k^T * scale) v, non-causal, per (batch, head).
+
+    q, k, v: bf16 CUDA [B, N, H, d] or [N, H, d] (any strides, last dim contiguous).
+    Returns o (same layout as q, new contiguous tensor unless `o` is given) and,
+    with return_lse, lse fp32 [B, H, N] (natural log)."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16_cuda(name, t)
+    squeeze = q.dim() == 3
+    if squeeze:
+        q, k, v = q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0)
+        if o is not None:
+            o = o.unsqueeze(0)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share a [B, N, H, d] shape")
+    B, N, H, d = q.shape
+    if o is None:
+        o = torch.empty((B, N, H, d), dtype=q.dtype, device=q.device)
+    _require_bf16_cuda("o", o)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if return_lse else None
+    st = lambda t: _I64_3(t.stride(0), t.stride(1), t.stride(2))
+    _check("h3attn_fwd", library().h3attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, N, H, d, st(q), st(k), st(v), st(o),
+        float(softmax_scale or 0.0), _ptr(lse), _stream_handle(stream)))
+    out = o.squeeze(0) if squeeze else o
+    if return_lse:
+        return out, (lse.squeeze(0) if squeeze else lse)
+    return out
+
+
+def attention_varlen(q, k, v, cu_seqlens, max_seqlen: int, o=None,
+                     softmax_scale: Optional[float] = None, return_lse: bool = False, stream=None):
+    """Attention over ragged sequences packed along tokens.
+
+    q, k, v: bf16 CUDA [total, H, d]; cu_seqlens: CUDA int32 [nseq + 1].
+    Returns o [total, H, d] and, with return_lse, lse fp32 [H, total]."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16_cuda(name, t)
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share a [total, H, d] shape")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or not cu_seqlens.is_contiguous():
+        raise TypeError("cu_seqlens must be a contiguous CUDA int32 tensor")
+    total, H, d = q.shape
+    if o is None:
+        o = torch.empty((total, H, d), dtype=q.dtype, device=q.device)
+    _require_bf16_cuda("o", o)
+    lse = torch.empty((H, total), dtype=torch.float32, device=q.device) if return_lse else None
+    st = lambda t: _I64_2(t.stride(0), t.stride(1))
+    _check("h3attn_fwd_varlen", library().h3attn_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), cu_seqlens.numel() - 1, total,
+        int(max_seqlen), H, d, st(q), st(k), st(v), st(o), float(softmax_scale or 0.0), _ptr(lse),
+        _stream_handle(stream)))
+    return (o, lse) if return_lse else o

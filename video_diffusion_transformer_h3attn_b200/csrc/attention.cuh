@@ -1,0 +1,398 @@
+// attention.cuh -- non-causal flash attention forward on sm_100a tensor cores.
+//
+// Computes O = softmax(Q K^T * scale) V per (sequence, head) over a packed
+// token sequence, the dominant cost of the MiniMax-H3 DiT block ("Buyer
+// Questions Status", block composition: attention is the largest share of the
+// profiled block; "Open-H3-Regenerate-2K", Forward table: dense attention on
+// one B200).  Ragged batches follow "H3 Runtime Current State" (ragged
+// sequence parallelism): each cu_seqlens segment attends only to itself.
+//
+// Structure of one CTA (320 threads, one CTA per SM):
+//   * two 128-row query tiles Q0, Q1 of one (sequence, head), resident in smem;
+//   * warp 8 (one lane): TMA producer.  Loads Q0/Q1 once, then K_j and V_j
+//     tiles (128 keys x d) into a ring of smem slots, K and V alternating;
+//   * warp 9 (one lane): tcgen05 MMA issuer.  S_t = Q_t K_j^T into tensor memory
+//     (fp32, 128 columns per tile), then O_t += P_t V_j with P_t read from tensor
+//     memory where softmax wrote it over S_t;
+//   * warps 0-3 / 4-7: online softmax for Q0 / Q1, one thread per query row
+//     (= one tensor-memory lane).  Running max m in log2 units, p = 2^(s*c - m)
+//     with c = scale*log2(e), running sum l of the bf16-rounded P (the weights the
+//     PV product uses, so they normalise to exactly one); P stored into
+//     the S columns; O rescaled in tensor memory only when the max grows by more
+//     than 2^8 (until then p stays <= 256, harmless in fp32 and bf16);
+//   * epilogue by the softmax warps: O / l to bf16, rows past the sequence end
+//     are not stored; LSE = (m + log2 l) * ln 2.
+// While softmax works on S_0 the tensor core computes S_1 and the previous PV
+// products, so MMA and exponentials overlap.  Every barrier wait is bounded.
+//
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 after.
+// Shared memory: Q0, Q1 and kStages K/V slots, each 128 rows x d bf16 stored as
+// d/64 blocks of 128 rows x 128 bytes with the 128-byte swizzle TMA writes and
+// the MMA descriptors read (K-major for Q and K, MN-major for V).
+#pragma once
+
+#include <cuda.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace h3 {
+
+constexpr int kBM = 128;        // query rows per tile (tensor-memory lanes)
+constexpr int kBN = 128;        // keys per K/V tile
+constexpr int kQTiles = 2;      // query tiles per CTA
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kAttnThreads = 320;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+
+template <int D>
+struct AttnTraits {
+  static constexpr int kAtoms = D / 64;                      // 128-byte swizzle atoms along d
+  static constexpr int kAtomBytes = kBM * 128;               // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kAtoms * kAtomBytes;     // one Q, K or V tile
+  static constexpr int kStages = (D == 128) ? 4 : 8;         // K/V ring slots
+  static constexpr int kTiles = kQTiles + kStages;
+  static constexpr int kBarriers = 1 + 2 * kStages + 3 * kQTiles;
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kTiles * kTileBytes + 8 * kBarriers + 16;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(256 + kQTiles * D <= 512, "tensor memory budget");
+};
+
+struct AttnParams {
+  uint16_t* o;                // bf16 output
+  int64_t o_batch, o_tok, o_head;
+  float* lse;                 // may be null
+  const int32_t* cu_seqlens;  // ragged only
+  int32_t nseq;               // ragged only
+  int32_t n_heads;
+  int64_t seqlen;             // dense: tokens per sequence
+  int64_t total;              // ragged: total tokens (LSE row stride per head)
+  float scale_log2;           // softmax_scale * log2(e)
+  LaunchCtl ctl;
+};
+
+// Bounded wait that ignores the launch-failed flag (used to drain copies in flight).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_test(bar, parity)) {
+    if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+template <int D, bool kVarlen>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
+  using T = AttnTraits<D>;
+  constexpr int kS = T::kStages;
+  extern __shared__ uint8_t smem_raw[];
+
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw_addr);
+  const uint32_t sQ = base;
+  const uint32_t sKV = base + kQTiles * T::kTileBytes;
+  const uint32_t bars = base + T::kTiles * T::kTileBytes;
+  const uint32_t bar_q = bars;
+  auto bar_kv_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto bar_kv_empty = [&](int s) { return bars + 8u * (1 + kS + s); };
+  auto bar_s_full = [&](int t) { return bars + 8u * (1 + 2 * kS + t); };
+  auto bar_p_full = [&](int t) { return bars + 8u * (1 + 2 * kS + kQTiles + t); };
+  auto bar_o_done = [&](int t) { return bars + 8u * (1 + 2 * kS + 2 * kQTiles + t); };
+  volatile uint32_t* const slot_words =
+      reinterpret_cast<volatile uint32_t*>(base_ptr + T::kTiles * T::kTileBytes + 8 * T::kBarriers);
+  // slot_words[0] = tensor-memory base, [1] = work valid, [2] = sequence, [3] = query-pair index
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const LaunchCtl ctl = p.ctl;
+
+  // ---- work decode (CTA-uniform, published through shared memory) ----------------
+  if (threadIdx.x == 0) {
+    uint32_t valid = launch_failed(ctl) ? 0u : 1u;
+    uint32_t seq = 0, pair = blockIdx.x;
+    if (kVarlen && valid) {
+      valid = 0;
+      uint32_t x = blockIdx.x;
+      for (int s = 0; s < p.nseq; ++s) {
+        const int32_t n = p.cu_seqlens[s + 1] - p.cu_seqlens[s];
+        const uint32_t pairs = n > 0 ? static_cast<uint32_t>((n + kQTiles * kBM - 1) / (kQTiles * kBM)) : 0u;
+        if (x < pairs) {
+          valid = 1;
+          seq = static_cast<uint32_t>(s);
+          pair = x;
+          break;
+        }
+        x -= pairs;
+      }
+    }
+    slot_words[1] = valid;
+    slot_words[2] = seq;
+    slot_words[3] = pair;
+  }
+  __syncthreads();
+  if (slot_words[1] == 0) return;  // CTA-uniform
+
+  const int head = blockIdx.y;
+  int batch = 0;
+  int64_t seq_base = 0;  // first token of the sequence in the tensor's token dimension
+  int64_t seq_len;
+  if (kVarlen) {
+    const int s = static_cast<int>(slot_words[2]);
+    seq_base = p.cu_seqlens[s];
+    seq_len = static_cast<int64_t>(p.cu_seqlens[s + 1]) - seq_base;
+  } else {
+    batch = blockIdx.z;
+    seq_len = p.seqlen;
+  }
+  const int64_t q_row0 = static_cast<int64_t>(slot_words[3]) * (kQTiles * kBM);
+  const int nkv = static_cast<int>((seq_len + kBN - 1) / kBN);
+  const int kv_last_valid = static_cast<int>(seq_len - static_cast<int64_t>(nkv - 1) * kBN);
+
+  // ---- setup: barriers and tensor memory --------------------------------------------
+  if (warp == kLoadWarp && lane == 0) {
+    ptx::mbar_init(bar_q, 1);
+    for (int s = 0; s < kS; ++s) {
+      ptx::mbar_init(bar_kv_full(s), 1);
+      ptx::mbar_init(bar_kv_empty(s), 1);
+    }
+    for (int t = 0; t < kQTiles; ++t) {
+      ptx::mbar_init(bar_s_full(t), 1);
+      ptx::mbar_init(bar_p_full(t), 128);
+      ptx::mbar_init(bar_o_done(t), 1);
+    }
+    ptx::fence_mbarrier_init();
+    ptx::tma_prefetch_desc(&tm_q);
+    ptx::tma_prefetch_desc(&tm_k);
+    ptx::tma_prefetch_desc(&tm_v);
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(ptx::smem_u32(const_cast<uint32_t*>(slot_words)), T::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = slot_words[0];
+
+  if (warp == kLoadWarp) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      bool ok = true;
+      const int32_t y_seq = static_cast<int32_t>(seq_base);
+      ptx::mbar_arrive_expect_tx(bar_q, kQTiles * T::kTileBytes);
+      for (int t = 0; t < kQTiles; ++t)
+        for (int a = 0; a < T::kAtoms; ++a)
+          ptx::tma_load_4d(sQ + t * T::kTileBytes + a * T::kAtomBytes, &tm_q, bar_q, a * 64,
+                           y_seq + static_cast<int32_t>(q_row0) + t * kBM, head, batch);
+      uint32_t it = 0;
+      for (int j = 0; j < nkv && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int slot = static_cast<int>(it % kS);
+          const uint32_t use = it / kS;
+          if (use > 0 && !mbar_wait(bar_kv_empty(slot), (use - 1) & 1u, ctl)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(bar_kv_full(slot), T::kTileBytes);
+          const CUtensorMap* map = kv ? &tm_v : &tm_k;
+          for (int a = 0; a < T::kAtoms; ++a)
+            ptx::tma_load_4d(sKV + slot * T::kTileBytes + a * T::kAtomBytes, map, bar_kv_full(slot),
+                             a * 64, y_seq + j * kBN, head, batch);
+        }
+      }
+      if (ok) {
+        // tail: the MMA warp's last releases must land before the CTA's smem is reused
+        const uint32_t first = it > static_cast<uint32_t>(kS) ? it - kS : 0u;
+        for (uint32_t u = first; u < it && ok; ++u)
+          ok = mbar_wait(bar_kv_empty(static_cast<int>(u % kS)), (u / kS) & 1u, ctl);
+      }
+      if (!ok) {
+        // failure: let the copies already issued land before the CTA releases its smem
+        mbar_wait_for(bar_q, 0, 20000000ull);
+        const uint32_t first = it > static_cast<uint32_t>(kS) ? it - kS : 0u;
+        for (uint32_t u = first; u < it; ++u)
+          mbar_wait_for(bar_kv_full(static_cast<int>(u % kS)), (u / kS) & 1u, 20000000ull);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================ MMA issuer ==================================
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBM, D, true);
+      // Ring order of the producer: K_j is load 2j, V_j is load 2j+1.
+      auto slot_of = [](uint32_t u) { return static_cast<int>(u % kS); };
+      auto parity_of = [](uint32_t u) { return (u / kS) & 1u; };
+      // S_t = Q_t K^T for the K tile in ring slot `ks`
+      auto issue_s = [&](int t, int ks) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * T::kAtomBytes + (kk & 3) * 32;
+          const uint64_t da = ptx::sdesc_sw128(sQ + t * T::kTileBytes + koff, 16, 1024);
+          const uint64_t db = ptx::sdesc_sw128(sKV + ks * T::kTileBytes + koff, 16, 1024);
+          ptx::mma_ss(tmem + t * 128, da, db, kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(bar_s_full(t));
+      };
+      // O_t += P_t V for the V tile in ring slot `vs`
+      auto issue_pv = [&](int t, int vs, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t db =
+              ptx::sdesc_sw128(sKV + vs * T::kTileBytes + kk * 16 * 128, T::kAtomBytes, 1024);
+          ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, kIdescPV,
+                      (!first || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(bar_o_done(t));
+      };
+
+      bool ok = mbar_wait(bar_q, 0, ctl) && mbar_wait(bar_kv_full(slot_of(0)), parity_of(0), ctl);
+      if (ok) {
+        ptx::tc_fence_after();
+        for (int t = 0; t < kQTiles; ++t) issue_s(t, slot_of(0));
+        ptx::mma_commit(bar_kv_empty(slot_of(0)));
+      }
+      // Skewed schedule: PV_t(j) is followed at once by S_t(j+1), so the tensor
+      // core always has the other tile's work while one softmax group runs.
+      for (int j = 0; j < nkv && ok; ++j) {
+        const uint32_t uv = 2u * j + 1u, uk = 2u * j + 2u;
+        const bool has_next = j + 1 < nkv;
+        if (!mbar_wait(bar_kv_full(slot_of(uv)), parity_of(uv), ctl)) { ok = false; break; }
+        if (has_next && !mbar_wait(bar_kv_full(slot_of(uk)), parity_of(uk), ctl)) { ok = false; break; }
+        for (int t = 0; t < kQTiles; ++t) {
+          if (!mbar_wait(bar_p_full(t), static_cast<uint32_t>(j) & 1u, ctl)) { ok = false; break; }
+          ptx::tc_fence_after();
+          issue_pv(t, slot_of(uv), j == 0);
+          if (t == kQTiles - 1) ptx::mma_commit(bar_kv_empty(slot_of(uv)));
+          if (has_next) issue_s(t, slot_of(uk));
+        }
+        if (!ok) break;
+        if (has_next) ptx::mma_commit(bar_kv_empty(slot_of(uk)));
+      }
+    }
+  } else {
+    // ============================ softmax + epilogue ==============================
+    const int t = warp >> 2;        // query tile
+    const int quarter = warp & 3;   // tensor-memory lane quarter of this warp
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const float c = p.scale_log2;
+    float m = -INFINITY;  // running max of s*c (log2 units), possibly stale by < 8
+    float l = 0.0f;       // running sum of 2^(s*c - m)
+    bool ok = true;
+
+    for (int j = 0; j < nkv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(t), static_cast<uint32_t>(j) & 1u, ctl));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tS + q * 32, sr[q]);
+      ptx::tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(sr[q][i]);
+      if (j == nkv - 1 && kv_last_valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= kv_last_valid) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+      const float cand = mx * c;
+      const bool grow = cand > m + kRescaleThreshold;
+      const float alpha = grow ? ptx::ex2_approx(m - cand) : 1.0f;
+      if (grow) m = cand;
+      l *= alpha;
+      // P = 2^(s*c - m), rounded to bf16, written over S in two halves of 64 keys
+      float sum = 0.0f;
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ptx::ex2_approx(fmaf(s[64 * hlf + 2 * i], c, -m));
+          const float p1 = ptx::ex2_approx(fmaf(s[64 * hlf + 2 * i + 1], c, -m));
+          pk[i] = ptx::pack_bf16x2(p0, p1);
+          // the row sum takes the rounded weights the PV product uses, so the
+          // normalised weights sum to one exactly
+          sum += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u);
+        }
+        ptx::tmem_st32(tS + hlf * 32, pk);
+      }
+      l += sum;
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_t(j-1) is final once S_t(j) has landed (the tensor core runs in issue
+        // order); the explicit wait keeps that visible.  Rescale it in place.
+        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(t), static_cast<uint32_t>(j - 1) & 1u, ctl));
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t orr[32];
+          ptx::tmem_ld32(tO + q * 32, orr);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          ptx::tmem_st32(tO + q * 32, orr);
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar_p_full(t));
+    }
+
+    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(t), static_cast<uint32_t>(nkv - 1) & 1u, ctl));
+    }
+    if (ok) {
+      ptx::tc_fence_after();
+      const int64_t row = q_row0 + t * kBM + quarter * 32 + lane;  // within the sequence
+      const bool valid = row < seq_len;
+      const float inv_l = 1.0f / l;
+      uint16_t* orow = p.o + static_cast<int64_t>(batch) * p.o_batch + (seq_base + row) * p.o_tok +
+                       static_cast<int64_t>(head) * p.o_head;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t orr[32];
+        ptx::tmem_ld32(tO + q * 32, orr);
+        ptx::tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = ptx::pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr) {
+        const float v = (m + log2f(l)) * 0.69314718055994530942f;
+        if (kVarlen) {
+          p.lse[static_cast<int64_t>(head) * p.total + seq_base + row] = v;
+        } else {
+          p.lse[(static_cast<int64_t>(batch) * p.n_heads + head) * p.seqlen + row] = v;
+        }
+      }
+    }
+  }
+
+  // ---- teardown: every thread arrives here, then the allocating warp frees TMEM ----
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, T::kTmemCols);
+  }
+}
+
+}  // namespace h3

@@ -1,0 +1,60 @@
+// common.cuh -- shared pieces of the h3attn kernels: the device error word and
+// bounded mbarrier waits.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace h3 {
+
+// Error bits recorded by kernels in the device error word.
+enum : uint32_t {
+  kErrTimeout = 1u,  // a bounded wait gave up
+};
+
+// Device error word: [0] = sticky error bits, [1] = id of the last launch that
+// failed (lets the other CTAs of that launch stop early without affecting later
+// launches).  Lives in the library module (the library is one translation
+// unit, so this is its only definition); read by h3attn_device_status().
+__device__ uint32_t g_error_word[2];
+
+// Longest a thread waits on one barrier phase before declaring the launch failed.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+struct LaunchCtl {
+  uint32_t launch_id;  // distinct per host call, never 0
+};
+
+__device__ __forceinline__ bool launch_failed(const LaunchCtl& ctl) {
+  return *reinterpret_cast<volatile uint32_t*>(&g_error_word[1]) == ctl.launch_id;
+}
+
+__device__ __forceinline__ void report_failure(const LaunchCtl& ctl, uint32_t bits) {
+  atomicOr(&g_error_word[0], bits);
+  atomicExch(&g_error_word[1], ctl.launch_id);
+}
+
+// Wait until the phase of `bar` with parity `parity` completes.  Returns false
+// (and records a timeout) after kWaitLimitNs, or early if another CTA of this
+// launch already failed.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, LaunchCtl ctl) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_test(bar, parity)) return true;
+    if ((it & 1023u) == 0) {
+      if (launch_failed(ctl)) return false;
+      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+        report_failure(ctl, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const LaunchCtl& ctl) {
+  if (ptx::mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, ctl);
+}
+
+}  // namespace h3

@@ -1,0 +1,337 @@
+// h3attn_api.cu -- the C ABI declared in include/h3attn.h: argument checks,
+// TMA tensor-map encoding, launch configuration, and the device error word.
+//
+// The whole library is this one translation unit (the kernels come in through
+// the headers), so it needs no relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "h3attn.h"
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "prologue.cuh"
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+
+thread_local char t_last_error[512] = "";
+
+h3attn_status fail(h3attn_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+h3attn_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(H3ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
+
+std::atomic<uint32_t> g_launch_counter{0};
+uint32_t next_launch_id() {
+  uint32_t id;
+  do {
+    id = g_launch_counter.fetch_add(1, std::memory_order_relaxed) + 1u;
+  } while (id == 0u);
+  return id;
+}
+
+// ---- driver entry point for cuTensorMapEncodeTiled (no link against libcuda) ----------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+  });
+  return fn;
+}
+
+// A bf16 [B][N][H][D] view (token-major) as a 4D tensor map with 128-row x 64-element
+// boxes and 128-byte swizzle.  Token rows outside [0, N) read as zeros.
+h3attn_status make_map(CUtensorMap* map, const void* ptr, int d, int64_t n_tok, int n_heads,
+                       int64_t n_batch, int64_t s_tok, int64_t s_head, int64_t s_batch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(H3ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n_tok),
+                        static_cast<cuuint64_t>(n_heads), static_cast<cuuint64_t>(n_batch)};
+  if (n_batch == 1) s_batch = s_tok;  // extent 1: the stride is never used
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s_tok) * 2, static_cast<cuuint64_t>(s_head) * 2,
+                           static_cast<cuuint64_t>(s_batch) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(h3::kBM), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(H3ATTN_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return H3ATTN_OK;
+}
+
+// Per-device one-time kernel attributes (dynamic shared memory opt-in).
+template <typename K>
+cudaError_t ensure_smem_attr(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D, bool kVarlen>
+h3attn_status launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                               const h3::AttnParams& prm, dim3 grid, cudaStream_t stream) {
+  using T = h3::AttnTraits<D>;
+  auto kernel = h3::attn_fwd_kernel<D, kVarlen>;
+  cudaError_t e = ensure_smem_attr(kernel, T::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
+  kernel<<<grid, h3::kAttnThreads, T::kSmemBytes, stream>>>(mq, mk, mv, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return H3ATTN_OK;
+}
+
+h3attn_status check_common(const void* q, const void* k, const void* v, void* o, int32_t n_heads,
+                           int32_t head_dim) {
+  if (!q || !k || !v || !o) return fail(H3ATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (n_heads <= 0 || n_heads > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "n_heads must be in [1, 65535]");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(H3ATTN_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(H3ATTN_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  return H3ATTN_OK;
+}
+
+h3attn_status check_strides(const int64_t* s, int n, const char* name) {
+  if (!s) return fail(H3ATTN_ERR_INVALID_ARG, "%s strides are null", name);
+  for (int i = 0; i < n; ++i) {
+    if (s[i] <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "%s stride %d must be positive", name, i);
+    if (s[i] % 8 != 0) return fail(H3ATTN_ERR_MISALIGNED, "%s stride %d not a multiple of 8 elements", name, i);
+    if (s[i] >= (int64_t(1) << 38)) return fail(H3ATTN_ERR_UNSUPPORTED, "%s stride %d too large", name, i);
+  }
+  return H3ATTN_OK;
+}
+
+float resolve_scale(float scale, int d) {
+  const float s = scale > 0.0f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  return static_cast<float>(static_cast<double>(s) * 1.4426950408889634074);
+}
+
+}  // namespace
+
+extern "C" {
+
+int h3attn_version(void) { return kVersion; }
+
+const char* h3attn_status_string(int status) {
+  switch (status) {
+    case H3ATTN_OK: return "ok";
+    case H3ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case H3ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case H3ATTN_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case H3ATTN_ERR_CUDA: return "CUDA error";
+    case H3ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    default: return "unknown status";
+  }
+}
+
+const char* h3attn_last_error(void) { return t_last_error; }
+
+int h3attn_device_status(void* stream, int clear) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t word[2] = {0, 0};
+  e = cudaMemcpyFromSymbol(word, h3::g_error_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (clear) {
+    const uint32_t zero[2] = {0, 0};
+    e = cudaMemcpyToSymbol(h3::g_error_word, zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  }
+  if (word[0] & h3::kErrTimeout)
+    return fail(H3ATTN_ERR_DEVICE_TIMEOUT, "a kernel timed out on an internal barrier (launch %u)", word[1]);
+  return H3ATTN_OK;
+}
+
+h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, void* k_out,
+                              int64_t n_tokens, int32_t n_heads, int32_t head_dim,
+                              int64_t in_tok_stride, int64_t in_head_stride,
+                              int64_t out_tok_stride, int64_t out_head_stride,
+                              const void* gamma_q, const void* gamma_k, double eps,
+                              const int32_t* pos, const uint8_t* kind,
+                              int32_t sec_t, int32_t sec_h, int32_t sec_w, double theta,
+                              void* stream) {
+  if (!q_in || !k_in || !q_out || !k_out) return fail(H3ATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (n_tokens < 0) return fail(H3ATTN_ERR_INVALID_ARG, "n_tokens must be >= 0");
+  if (n_heads <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "n_heads must be positive");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(H3ATTN_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(q_out) || !aligned16(k_out) ||
+      (gamma_q && !aligned16(gamma_q)) || (gamma_k && !aligned16(gamma_k)))
+    return fail(H3ATTN_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  const int64_t strides[4] = {in_tok_stride, in_head_stride, out_tok_stride, out_head_stride};
+  h3attn_status st = check_strides(strides, 4, "prologue");
+  if (st != H3ATTN_OK) return st;
+  if (!(eps >= 0.0) || !std::isfinite(eps)) return fail(H3ATTN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+
+  h3::PrologueParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (pos) {
+    if (!kind) return fail(H3ATTN_ERR_INVALID_ARG, "kind is required with pos");
+    if (sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t | sec_h | sec_w) & 1 || sec_t + sec_h + sec_w != head_dim)
+      return fail(H3ATTN_ERR_INVALID_ARG, "sections %d/%d/%d must be even and sum to head_dim %d", sec_t,
+                  sec_h, sec_w, head_dim);
+    if (!(theta > 0.0) || !std::isfinite(theta)) return fail(H3ATTN_ERR_INVALID_ARG, "theta must be > 0");
+    // rotary tables: pair p of the 3D layout belongs to section ax at pair index i inside it
+    const int widths[3] = {sec_t, sec_h, sec_w};
+    int pair = 0;
+    for (int ax = 0; ax < 3; ++ax) {
+      for (int i = 0; i < widths[ax] / 2; ++i, ++pair) {
+        prm.rope.axis_3d[pair] = static_cast<uint8_t>(ax);
+        prm.rope.inv_freq_3d[pair] = std::exp(-(2.0 * i / widths[ax]) * std::log(theta));
+      }
+    }
+    for (int i = 0; i < head_dim / 2; ++i)
+      prm.rope.inv_freq_1d[i] = std::exp(-(2.0 * i / head_dim) * std::log(theta));
+  }
+  if (n_tokens == 0) return H3ATTN_OK;
+  prm.q_in = static_cast<const uint16_t*>(q_in);
+  prm.k_in = static_cast<const uint16_t*>(k_in);
+  prm.q_out = static_cast<uint16_t*>(q_out);
+  prm.k_out = static_cast<uint16_t*>(k_out);
+  prm.n_tokens = n_tokens;
+  prm.in_tok = in_tok_stride;
+  prm.in_head = in_head_stride;
+  prm.out_tok = out_tok_stride;
+  prm.out_head = out_head_stride;
+  prm.gamma_q = static_cast<const uint16_t*>(gamma_q);
+  prm.gamma_k = static_cast<const uint16_t*>(gamma_k);
+  prm.pos = pos;
+  prm.kind = kind;
+  prm.n_heads = n_heads;
+  prm.eps = static_cast<float>(eps);
+
+  constexpr int kThreads = 256;
+  constexpr int kTokensPerBlock = kThreads / 32;
+  const int64_t blocks = (n_tokens + kTokensPerBlock - 1) / kTokensPerBlock;
+  if (blocks > 0x7FFFFFFF) return fail(H3ATTN_ERR_UNSUPPORTED, "too many tokens");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128) {
+    h3::prologue_kernel<128><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(prm);
+  } else {
+    h3::prologue_kernel<64><<<static_cast<unsigned>(blocks), kThreads, 0, s>>>(prm);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+  return H3ATTN_OK;
+}
+
+h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, int32_t batch,
+                         int64_t seqlen, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
+                         const int64_t k_strides[3], const int64_t v_strides[3],
+                         const int64_t o_strides[3], float softmax_scale, float* lse, void* stream) {
+  h3attn_status st = check_common(q, k, v, o, n_heads, head_dim);
+  if (st != H3ATTN_OK) return st;
+  if (batch <= 0 || batch > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "batch must be in [1, 65535]");
+  if (seqlen <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be positive");
+  if (seqlen > (int64_t(1) << 30)) return fail(H3ATTN_ERR_UNSUPPORTED, "seqlen too large");
+  if ((st = check_strides(q_strides, 3, "q")) != H3ATTN_OK) return st;
+  if ((st = check_strides(k_strides, 3, "k")) != H3ATTN_OK) return st;
+  if ((st = check_strides(v_strides, 3, "v")) != H3ATTN_OK) return st;
+  if ((st = check_strides(o_strides, 3, "o")) != H3ATTN_OK) return st;
+  if (!std::isfinite(softmax_scale)) return fail(H3ATTN_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(H3ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, head_dim, seqlen, n_heads, batch, q_strides[1], q_strides[2], q_strides[0])) != H3ATTN_OK) return st;
+  if ((st = make_map(&mk, k, head_dim, seqlen, n_heads, batch, k_strides[1], k_strides[2], k_strides[0])) != H3ATTN_OK) return st;
+  if ((st = make_map(&mv, v, head_dim, seqlen, n_heads, batch, v_strides[1], v_strides[2], v_strides[0])) != H3ATTN_OK) return st;
+
+  h3::AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.o = static_cast<uint16_t*>(o);
+  prm.o_batch = o_strides[0];
+  prm.o_tok = o_strides[1];
+  prm.o_head = o_strides[2];
+  prm.lse = lse;
+  prm.n_heads = n_heads;
+  prm.seqlen = seqlen;
+  prm.total = seqlen;
+  prm.scale_log2 = resolve_scale(softmax_scale, head_dim);
+  prm.ctl.launch_id = next_launch_id();
+
+  const int64_t pairs = (seqlen + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM);
+  dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return head_dim == 128 ? launch_attention<128, false>(mq, mk, mv, prm, grid, s)
+                         : launch_attention<64, false>(mq, mk, mv, prm, grid, s);
+}
+
+h3attn_status h3attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
+                                const int32_t* cu_seqlens, int32_t nseq, int64_t total_tokens,
+                                int32_t max_seqlen, int32_t n_heads, int32_t head_dim,
+                                const int64_t q_strides[2], const int64_t k_strides[2],
+                                const int64_t v_strides[2], const int64_t o_strides[2],
+                                float softmax_scale, float* lse, void* stream) {
+  h3attn_status st = check_common(q, k, v, o, n_heads, head_dim);
+  if (st != H3ATTN_OK) return st;
+  if (!cu_seqlens) return fail(H3ATTN_ERR_INVALID_ARG, "cu_seqlens is null");
+  if (nseq <= 0 || nseq > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "nseq must be in [1, 65535]");
+  if (total_tokens <= 0 || total_tokens > (int64_t(1) << 30))
+    return fail(H3ATTN_ERR_INVALID_ARG, "total_tokens must be in [1, 2^30]");
+  if (max_seqlen <= 0 || max_seqlen > total_tokens)
+    return fail(H3ATTN_ERR_INVALID_ARG, "max_seqlen must be in [1, total_tokens]");
+  if ((st = check_strides(q_strides, 2, "q")) != H3ATTN_OK) return st;
+  if ((st = check_strides(k_strides, 2, "k")) != H3ATTN_OK) return st;
+  if ((st = check_strides(v_strides, 2, "v")) != H3ATTN_OK) return st;
+  if ((st = check_strides(o_strides, 2, "o")) != H3ATTN_OK) return st;
+  if (!std::isfinite(softmax_scale)) return fail(H3ATTN_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(H3ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, head_dim, total_tokens, n_heads, 1, q_strides[0], q_strides[1], 0)) != H3ATTN_OK) return st;
+  if ((st = make_map(&mk, k, head_dim, total_tokens, n_heads, 1, k_strides[0], k_strides[1], 0)) != H3ATTN_OK) return st;
+  if ((st = make_map(&mv, v, head_dim, total_tokens, n_heads, 1, v_strides[0], v_strides[1], 0)) != H3ATTN_OK) return st;
+
+  h3::AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.o = static_cast<uint16_t*>(o);
+  prm.o_batch = 0;
+  prm.o_tok = o_strides[0];
+  prm.o_head = o_strides[1];
+  prm.lse = lse;
+  prm.cu_seqlens = cu_seqlens;
+  prm.nseq = nseq;
+  prm.n_heads = n_heads;
+  prm.seqlen = max_seqlen;
+  prm.total = total_tokens;
+  prm.scale_log2 = resolve_scale(softmax_scale, head_dim);
+  prm.ctl.launch_id = next_launch_id();
+
+  // upper bound on query-tile pairs: each sequence wastes at most one partial pair
+  const int64_t pairs = (total_tokens + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM) + nseq;
+  dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), 1);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return head_dim == 128 ? launch_attention<128, true>(mq, mk, mv, prm, grid, s)
+                         : launch_attention<64, true>(mq, mk, mv, prm, grid, s);
+}
+
+}  // extern "C"
