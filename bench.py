@@ -378,6 +378,51 @@ def run_gpu(args):
     return 0
 
 
+def run_kernel_only(args):
+    """W + K launches of one kernel on one workload and nothing else (for ncu captures)."""
+    import torch
+
+    import video_diffusion_transformer_h3attn_b200 as h3
+    from video_diffusion_transformer_h3attn_b200 import inputs
+
+    w = inputs.workload(args.workload)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+    q, k, v = bf16(w.q), bf16(w.k), bf16(w.v)
+    out = torch.empty_like(q)
+    if args.kernel_only == "prologue":
+        g = (bf16(w.gamma_q), bf16(w.gamma_k)) if w.gamma_q is not None else (None, None)
+        pos = torch.from_numpy(w.pos).cuda() if w.pos is not None else None
+        kind = torch.from_numpy(w.kind).cuda() if w.kind is not None else None
+        kout = torch.empty_like(k)
+        run = lambda: h3.prologue(q, k, out, kout, g[0], g[1], w.eps, pos, kind, w.sections, w.theta)
+        unit = 4.0 * w.total * w.n_heads * w.head_dim * 2 / 1e9  # GB per launch
+    elif len(w.seqlens) > 1:
+        cu = torch.from_numpy(w.cu_seqlens).cuda()
+        run = lambda: h3.attention_varlen(q, k, v, cu, max(w.seqlens), out)
+        unit = w.attention_flops() / 1e12
+    else:
+        run = lambda: h3.attention(q, k, v, out)
+        unit = w.attention_flops() / 1e12
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    h3.device_status()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"kernel": args.kernel_only, "workload": args.workload, "ms": ms,
+                      "rate": unit / (ms * 1e-3),
+                      "rate_unit": "GB/s" if args.kernel_only == "prologue" else "TFLOP/s"}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -385,7 +430,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["h3attn", "reference"], default="h3attn")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload for --kernel-only runs (tiny, small, joint, 2k, ragged)")
+    ap.add_argument("--kernel-only", choices=["attention", "prologue"],
+                    help="launch only this kernel W + K times (profiling runs)")
     args = ap.parse_args()
+    if args.kernel_only:
+        return run_kernel_only(args)
     if args.warmup < 3 and args.impl == "h3attn":
         print("note: raising --warmup to 3", file=sys.stderr)
         args.warmup = 3

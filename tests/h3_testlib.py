@@ -4,10 +4,12 @@ comparing against the fp64 oracle, and the tolerances.
 Tolerances (written here once, used by every parity test):
   prologue   every output within 1 bf16 ulp of the correctly rounded oracle value
              (|ordered(bits_gpu) - ordered(bf16(oracle))| <= 1);
-  attention  mean |o_gpu - o_ref| <= 1e-3 and, element by element,
-             |o_gpu - o_ref| - ulp_bf16(o_ref)/2 <= 1e-2: the max-abs bound of 1e-2
-             applies to the error beyond the half-ulp that storing the exact value as
-             bf16 costs by itself (for |o| >= 4 that half ulp alone exceeds 1e-2);
+  attention  the error beyond the half-ulp that storing the exact value as bf16
+             costs by itself, e = max(0, |o_gpu - o_ref| - ulp_bf16(o_ref)/2), has
+             max <= 1e-2 and mean <= 1e-3 (for |o| >= 4 that half ulp alone exceeds
+             1e-2; for rows over a few keys |o| ~ 1 and it dominates the mean);
+             strict=True (the five named workloads) also requires the plain
+             max |o_gpu - o_ref| <= 1e-2 and mean <= 1e-3;
   lse        |lse_gpu - lse_ref| <= 1e-3 (fp32 output).
 """
 from __future__ import annotations
@@ -59,16 +61,20 @@ def check_prologue(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str) -> dic
     return stats
 
 
-def check_attention(o_gpu: np.ndarray, o_ref: np.ndarray, what: str, lse_gpu=None, lse_ref=None) -> dict:
+def check_attention(o_gpu: np.ndarray, o_ref: np.ndarray, what: str, lse_gpu=None, lse_ref=None,
+                    strict: bool = False) -> dict:
     o_gpu = np.asarray(o_gpu, dtype=np.float64)
     err = np.abs(o_gpu - o_ref)
-    excess = err - bf16_half_ulp(o_ref)
+    excess = np.maximum(err - bf16_half_ulp(o_ref), 0.0)
     stats = {"max_abs": float(err.max()), "mean_abs": float(err.mean()),
-             "max_excess": float(excess.max())}
+             "max_excess": float(excess.max()), "mean_excess": float(excess.mean())}
     assert np.all(np.isfinite(o_gpu)), "%s: non-finite output" % what
     assert stats["max_excess"] <= ATTN_MAX_ABS, "%s: %s at %s" % (
         what, stats, np.unravel_index(int(np.argmax(excess)), excess.shape))
-    assert stats["mean_abs"] <= ATTN_MEAN_ABS, "%s: %s" % (what, stats)
+    assert stats["mean_excess"] <= ATTN_MEAN_ABS, "%s: %s" % (what, stats)
+    if strict:
+        assert stats["max_abs"] <= ATTN_MAX_ABS, "%s (strict): %s" % (what, stats)
+        assert stats["mean_abs"] <= ATTN_MEAN_ABS, "%s (strict): %s" % (what, stats)
     if lse_gpu is not None:
         le = np.abs(np.asarray(lse_gpu, dtype=np.float64) - lse_ref)
         stats["lse_max_abs"] = float(le.max())

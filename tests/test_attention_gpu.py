@@ -62,7 +62,7 @@ def test_tiny_full(h3, orc):
     w = inputs.workload("tiny")
     o, lse = _gpu_dense(h3, w.q, w.k, w.v)
     ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
-    check_attention(bf16_bits_to_f64(o), ro, "tiny", lse.T, rl)
+    check_attention(bf16_bits_to_f64(o), ro, "tiny", lse.T, rl, strict=True)
 
 
 def test_small_full(h3, orc):
@@ -70,7 +70,7 @@ def test_small_full(h3, orc):
     q, k = _qk(orc, w)
     o, lse = _gpu_dense(h3, q, k, w.v)
     ro, rl = orc.attention(q, k, w.v, w.cu_seqlens)
-    check_attention(bf16_bits_to_f64(o), ro, "small", lse.T, rl)
+    check_attention(bf16_bits_to_f64(o), ro, "small", lse.T, rl, strict=True)
 
 
 @pytest.mark.parametrize("name,n_rows", [("joint", 384), ("2k", 160)])
@@ -80,7 +80,7 @@ def test_large_sampled(h3, orc, name, n_rows):
     o, lse = _gpu_dense(h3, q, k, w.v)
     rows = inputs.sample_rows(w.cu_seqlens, n_rows, seed=w.seed + 1000)
     ro, rl = orc.attention(q, k, w.v, w.cu_seqlens, rows=rows)
-    check_attention(bf16_bits_to_f64(o[rows]), ro, name, lse.T[rows], rl)
+    check_attention(bf16_bits_to_f64(o[rows]), ro, name, lse.T[rows], rl, strict=True)
 
 
 def test_ragged_sampled(h3, orc):
@@ -89,7 +89,7 @@ def test_ragged_sampled(h3, orc):
     o, lse = _gpu_varlen(h3, q, k, w.v, w.cu_seqlens)
     rows = inputs.sample_rows(w.cu_seqlens, 384, seed=w.seed + 1000)
     ro, rl = orc.attention(q, k, w.v, w.cu_seqlens, rows=rows)
-    check_attention(bf16_bits_to_f64(o[rows]), ro, "ragged", lse.T[rows], rl)
+    check_attention(bf16_bits_to_f64(o[rows]), ro, "ragged", lse.T[rows], rl, strict=True)
 
 
 @pytest.mark.parametrize("n", [1, 2, 127, 128, 129, 255, 256, 257, 383, 640])

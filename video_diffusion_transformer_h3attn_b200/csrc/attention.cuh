@@ -17,11 +17,12 @@
 //   * warps 0-3 / 4-7: online softmax for Q0 / Q1, one thread per query row
 //     (= one tensor-memory lane).  Running max m in log2 units, p = 2^(s*c - m)
 //     with c = scale*log2(e), running sum l of the bf16-rounded P (the weights the
-//     PV product uses, so they normalise to exactly one); P stored into
+//     PV product uses, so they normalise to exactly one) and lx of the unrounded
+//     P (for the log-sum-exp); P stored into
 //     the S columns; O rescaled in tensor memory only when the max grows by more
 //     than 2^8 (until then p stays <= 256, harmless in fp32 and bf16);
 //   * epilogue by the softmax warps: O / l to bf16, rows past the sequence end
-//     are not stored; LSE = (m + log2 l) * ln 2.
+//     are not stored; LSE = (m + log2 lx) * ln 2.
 // While softmax works on S_0 the tensor core computes S_1 and the previous PV
 // products, so MMA and exponentials overlap.  Every barrier wait is bounded.
 //
@@ -282,7 +283,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tO = tmem + lane_off + 256 + t * D;
     const float c = p.scale_log2;
     float m = -INFINITY;  // running max of s*c (log2 units), possibly stale by < 8
-    float l = 0.0f;       // running sum of 2^(s*c - m)
+    float l = 0.0f;       // running sum of bf16(2^(s*c - m)): normalises O
+    float lx = 0.0f;      // running sum of 2^(s*c - m) in fp32: the log-sum-exp
     bool ok = true;
 
     for (int j = 0; j < nkv; ++j) {
@@ -311,8 +313,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float alpha = grow ? ptx::ex2_approx(m - cand) : 1.0f;
       if (grow) m = cand;
       l *= alpha;
+      lx *= alpha;
       // P = 2^(s*c - m), rounded to bf16, written over S in two halves of 64 keys
-      float sum = 0.0f;
+      float sum = 0.0f, sumx = 0.0f;
 #pragma unroll
       for (int hlf = 0; hlf < 2; ++hlf) {
         uint32_t pk[32];
@@ -321,13 +324,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const float p0 = ptx::ex2_approx(fmaf(s[64 * hlf + 2 * i], c, -m));
           const float p1 = ptx::ex2_approx(fmaf(s[64 * hlf + 2 * i + 1], c, -m));
           pk[i] = ptx::pack_bf16x2(p0, p1);
-          // the row sum takes the rounded weights the PV product uses, so the
-          // normalised weights sum to one exactly
+          // l sums the rounded weights the PV product uses (they normalise to one
+          // exactly); lx sums the unrounded ones for the log-sum-exp output
           sum += __uint_as_float(pk[i] << 16) + __uint_as_float(pk[i] & 0xFFFF0000u);
+          sumx += p0 + p1;
         }
         ptx::tmem_st32(tS + hlf * 32, pk);
       }
       l += sum;
+      lx += sumx;
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         // O_t(j-1) is final once S_t(j) has landed (the tensor core runs in issue
         // order); the explicit wait keeps that visible.  Rescale it in place.
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       if (valid && p.lse != nullptr) {
-        const float v = (m + log2f(l)) * 0.69314718055994530942f;
+        const float v = (m + log2f(lx)) * 0.69314718055994530942f;
         if (kVarlen) {
           p.lse[static_cast<int64_t>(head) * p.total + seq_base + row] = v;
         } else {

@@ -2,7 +2,7 @@
 //
 // The fused norm/RoPE step that feeds attention in the MiniMax-H3 DiT block
 // ("H3 Runtime Current State", Owned Performance Kernels: fused Q/K RMSNorm,
-// RoPE and layout work; "Buyer Questions Status", block composition: norm/RoPE
+// RoPE and layout work; "Buyer Questions: Current Evidence Status", block composition: norm/RoPE
 // share of the block).  The operation is stated in h3attn.h (h3attn_prologue).
 //
 // Work layout: one warp per token.  A row of head_dim bf16 values is 16 lanes x
