@@ -225,6 +225,17 @@ def profiled_traffic():
     return rec.get("dram_bytes_per_launch")
 
 
+def reduce_max(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (the job is as slow as its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -281,11 +292,7 @@ def run_gpu(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     # ---- device-resident timing ----
     for _ in range(args.warmup):

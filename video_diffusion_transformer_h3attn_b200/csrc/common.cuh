@@ -38,11 +38,15 @@ __device__ __forceinline__ void report_failure(const LaunchCtl& ctl, uint32_t bi
 // Wait until the phase of `bar` with parity `parity` completes.  Returns false
 // (and records a timeout) after kWaitLimitNs, or early if another CTA of this
 // launch already failed.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, LaunchCtl ctl) {
+// Each probe may suspend the thread for up to kSleepHintNs, so a waiting warp
+// neither spins nor takes issue slots from the warps doing the work.
+constexpr uint32_t kSleepHintNs = 1000000;  // 1 ms
+
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, LaunchCtl ctl) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (ptx::mbar_test(bar, parity)) return true;
-    if ((it & 1023u) == 0) {
+    if (ptx::mbar_test_sleep(bar, parity, kSleepHintNs)) return true;
+    if ((it & 15u) == 0) {
       if (launch_failed(ctl)) return false;
       if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
         report_failure(ctl, kErrTimeout);

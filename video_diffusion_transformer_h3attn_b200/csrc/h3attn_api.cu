@@ -99,7 +99,7 @@ template <int D, bool kVarlen>
 h3attn_status launch_attention(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const h3::AttnParams& prm, dim3 grid, cudaStream_t stream) {
   using T = h3::AttnTraits<D>;
-  auto kernel = h3::attn_fwd_kernel<D, kVarlen>;
+  auto kernel = prm.lse ? h3::attn_fwd_kernel<D, kVarlen, true> : h3::attn_fwd_kernel<D, kVarlen, false>;
   cudaError_t e = ensure_smem_attr(kernel, T::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attention)");
   kernel<<<grid, h3::kAttnThreads, T::kSmemBytes, stream>>>(mq, mk, mv, prm);
