@@ -17,18 +17,17 @@
 //     tensor memory, where softmax wrote it over S_t.  Order per step j:
 //     PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so the tensor core always holds the
 //     other tile's work while one softmax group runs;
-//   * warps 0-7 / 8-15 -- online softmax of Q0 / Q1.  Each query row (= one
-//     tensor-memory lane) is shared by two threads in two warps of the same lane
-//     quarter, one per 64-key half, so every scheduler runs two warps of the
-//     active tile.  The halves trade their row maxima through shared memory
-//     each step (an mbarrier orders it) and agree on one running max m (log2
-//     units, may lag the true max by < 8 so that P <= 256 and O is rescaled
-//     rarely); p = 2^(s*c - m) with c = scale*log2(e); P rounded to bf16 and
-//     stored over S; l sums the rounded weights the PV product uses (they
-//     normalise to exactly one), lx the unrounded ones (log-sum-exp);
-//   * epilogue by the softmax warps: the halves add their row sums, each stores
-//     its half of O / l as bf16; rows past the sequence end are not stored;
-//     LSE = (m + log2 lx) * ln 2.
+//   * warps 0-7 / 8-15 -- online softmax of Q0 / Q1.  A warp owns 16 tensor-
+//     memory lanes and reads them with the 16x256b shape, so each query row's
+//     128 scores sit in four threads of one warp (32 each): row maxima and sums
+//     are two shuffles away, and two warps per scheduler work on each tile.  The
+//     running max m (log2 units) may lag the true max by < 8, so P <= 256 and O
+//     is rescaled in tensor memory only when the max grows by more;
+//     p = 2^(s*c - m) with c = scale*log2(e), rounded to bf16 and stored over S
+//     with the 16x128b shape; l sums the rounded weights the PV product uses
+//     (they normalise to exactly one), lx the unrounded ones (log-sum-exp);
+//   * epilogue by the softmax warps: O / l as bf16 (rows past the sequence end
+//     are not stored); LSE = (m + log2 lx) * ln 2.
 // Every barrier wait is bounded (common.cuh).
 //
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 after.
@@ -63,11 +62,9 @@ struct AttnTraits {
   static constexpr int kTileBytes = kAtoms * kAtomBytes;     // one Q, K or V tile
   static constexpr int kStages = (D == 128) ? 4 : 8;         // K/V ring slots
   static constexpr int kTiles = kQTiles + kStages;
-  // barriers: q, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], xch[2][4]
-  static constexpr int kBarriers = 1 + 2 * kStages + 3 * kQTiles + kQTiles * 4;
-  static constexpr int kXchBytes = 2 * kQTiles * 2 * kBM * 4;  // [parity][tile][half][row] fp32
-  static constexpr int kSmemBytes =
-      1024 /*alignment slack*/ + kTiles * kTileBytes + kXchBytes + 8 * kBarriers + 16;
+  // barriers: q, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2]
+  static constexpr int kBarriers = 1 + 2 * kStages + 3 * kQTiles;
+  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kTiles * kTileBytes + 8 * kBarriers + 16;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(256 + kQTiles * D <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -138,17 +135,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* const base_ptr = smem_raw + (base - raw_addr);
   const uint32_t sQ = base;
   const uint32_t sKV = base + kQTiles * T::kTileBytes;
-  float* const xch = reinterpret_cast<float*>(base_ptr + T::kTiles * T::kTileBytes);
-  const uint32_t bars = base + T::kTiles * T::kTileBytes + T::kXchBytes;
+  const uint32_t bars = base + T::kTiles * T::kTileBytes;
   const uint32_t bar_q = bars;
   auto bar_kv_full = [&](int s) { return bars + 8u * (1 + s); };
   auto bar_kv_empty = [&](int s) { return bars + 8u * (1 + kS + s); };
   auto bar_s_full = [&](int t) { return bars + 8u * (1 + 2 * kS + t); };
   auto bar_p_full = [&](int t) { return bars + 8u * (1 + 2 * kS + kQTiles + t); };
   auto bar_o_done = [&](int t) { return bars + 8u * (1 + 2 * kS + 2 * kQTiles + t); };
-  auto bar_xch = [&](int t, int q) { return bars + 8u * (1 + 2 * kS + 3 * kQTiles + 4 * t + q); };
-  volatile uint32_t* const slot_words = reinterpret_cast<volatile uint32_t*>(
-      base_ptr + T::kTiles * T::kTileBytes + T::kXchBytes + 8 * T::kBarriers);
+  volatile uint32_t* const slot_words =
+      reinterpret_cast<volatile uint32_t*>(base_ptr + T::kTiles * T::kTileBytes + 8 * T::kBarriers);
   // slot_words[0] = tensor-memory base, [1] = work valid, [2] = sequence, [3] = query-pair index
 
   const int warp = threadIdx.x >> 5;
@@ -206,9 +201,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int t = 0; t < kQTiles; ++t) {
       ptx::mbar_init(bar_s_full(t), 1);
-      ptx::mbar_init(bar_p_full(t), kSoftmaxWarps / kQTiles);
+      ptx::mbar_init(bar_p_full(t), kSoftmaxWarps / kQTiles);  // one arrival per warp of the tile
       ptx::mbar_init(bar_o_done(t), 1);
-      for (int q = 0; q < 4; ++q) ptx::mbar_init(bar_xch(t, q), 64);
     }
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tm_q);
@@ -301,6 +295,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ptx::mma_commit(bar_o_done(t));
       };
 
+      // Descriptor sets for one K = 128 block, built while the thread waits anyway,
+      // so each group of MMAs goes out back to back (d = 128: eight per group).
+      auto q_descs = [&](int t, uint64_t (&d)[8]) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          d[kk] = ptx::sdesc_make(q_lo0 + t * kTile16 + (((kk >> 2) * T::kAtomBytes + (kk & 3) * 32) >> 4), kHi);
+      };
+      auto k_descs = [&](int ks, uint64_t (&d)[8]) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          d[kk] = ptx::sdesc_make(k_lo0 + ks * kTile16 + (((kk >> 2) * T::kAtomBytes + (kk & 3) * 32) >> 4), kHi);
+      };
+      auto v_descs = [&](int vs, uint64_t (&d)[8]) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) d[kk] = ptx::sdesc_make(v_lo0 + vs * kTile16 + ((kk * 16 * 128) >> 4), kHi);
+      };
+      auto p_addrs = [&](int t, uint32_t (&a)[8]) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) a[kk] = tmem + t * 128 + kk * 8;
+      };
+
       bool ok = mbar_wait(bar_q, 0, ctl) && mbar_wait(bar_kv_full(slot_of(0)), parity_of(0), ctl);
       if (ok) {
         ptx::tc_fence_after();
@@ -311,15 +326,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t uv = 2u * j + 1u, uk = 2u * j + 2u;
         const bool has_next = j + 1 < nkv;
         if (!mbar_wait(bar_kv_full(slot_of(uv)), parity_of(uv), ctl)) { ok = false; break; }
-        for (int t = 0; t < kQTiles; ++t) {
-          if (!mbar_wait(bar_p_full(t), static_cast<uint32_t>(j) & 1u, ctl)) { ok = false; break; }
-          ptx::tc_fence_after();
-          issue_pv(t, slot_of(uv), j == 0);
-          if (t == kQTiles - 1) ptx::mma_commit(bar_kv_empty(slot_of(uv)));
-          if (has_next) {
-            // K_{j+1} is only needed here, after PV_t(j) has been issued
-            if (t == 0 && !mbar_wait(bar_kv_full(slot_of(uk)), parity_of(uk), ctl)) { ok = false; break; }
-            issue_s(t, slot_of(uk));
+        if constexpr (D == 128) {
+          uint64_t dv[8], dk[8], dq[8];
+          uint32_t ap[8];
+          v_descs(slot_of(uv), dv);
+          k_descs(slot_of(uk), dk);
+#pragma unroll
+          for (int t = 0; t < kQTiles; ++t) {
+            q_descs(t, dq);
+            p_addrs(t, ap);
+            if (!mbar_wait(bar_p_full(t), static_cast<uint32_t>(j) & 1u, ctl)) { ok = false; break; }
+            ptx::tc_fence_after();
+            ptx::mma_ts_x8(tmem + 256 + t * D, ap, dv, kIdescPV, j > 0 ? 1u : 0u);
+            ptx::mma_commit(bar_o_done(t));
+            if (t == kQTiles - 1) ptx::mma_commit(bar_kv_empty(slot_of(uv)));
+            if (has_next) {
+              // K_{j+1} is only needed here, after PV_t(j) has been issued
+              if (t == 0 && !mbar_wait(bar_kv_full(slot_of(uk)), parity_of(uk), ctl)) { ok = false; break; }
+              ptx::mma_ss_x8(tmem + t * 128, dq, dk, kIdescQK, 0u);
+              ptx::mma_commit(bar_s_full(t));
+            }
+          }
+        } else {
+          for (int t = 0; t < kQTiles; ++t) {
+            if (!mbar_wait(bar_p_full(t), static_cast<uint32_t>(j) & 1u, ctl)) { ok = false; break; }
+            ptx::tc_fence_after();
+            issue_pv(t, slot_of(uv), j == 0);
+            if (t == kQTiles - 1) ptx::mma_commit(bar_kv_empty(slot_of(uv)));
+            if (has_next) {
+              if (t == 0 && !mbar_wait(bar_kv_full(slot_of(uk)), parity_of(uk), ctl)) { ok = false; break; }
+              issue_s(t, slot_of(uk));
+            }
           }
         }
         if (!ok) break;
@@ -328,110 +365,136 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ============================ softmax + epilogue ==============================
-    const int t = warp >> 3;            // query tile
-    const int half = (warp >> 2) & 1;   // which 64 keys of each row this thread owns
-    const int quarter = warp & 3;       // tensor-memory lane quarter of this warp
-    const int row_in_tile = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;                         // S / P columns
-    const uint32_t tO = tmem + lane_off + 256 + t * D + half * (D / 2);    // this half of O
-    const uint32_t xbar = bar_xch(t, quarter);
-    constexpr int kParityStride = kQTiles * 2 * kBM;  // floats per exchange buffer
-    float* const xmine = xch + ((t * 2 + half) * kBM + row_in_tile);
-    float* const xpeer = xch + ((t * 2 + (half ^ 1)) * kBM + row_in_tile);
+    // Warps 0-7 serve tile 0 and warps 8-15 tile 1.  A warp owns 16 tensor-memory
+    // lanes (half of its lane quarter) and reads them with the 16x256b shape:
+    // thread t holds rows r0 = t/4 and r1 = t/4 + 8 of those 16, 32 keys each
+    // (columns 8k + 2(t%4) + {0,1}), so a row's 128 keys sit in 4 threads of the
+    // same warp and its max and sums are two shuffles away.
+    const int t = warp >> 3;                 // query tile
+    const int quarter = warp & 3;
+    const int lhalf = (warp >> 2) & 1;       // which 16 lanes of the quarter
+    const int cq = lane & 3;                 // column phase inside each 8-column chunk
+    const int lane0 = quarter * 32 + lhalf * 16;   // first tensor-memory lane of this warp
+    const int r0 = lane0 + (lane >> 2);      // this thread's two rows (tile-relative)
+    const int r1 = r0 + 8;
+    const uint32_t lane_off = static_cast<uint32_t>(lane0) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
     const float c = p.scale_log2;
-    float m = -INFINITY;  // running max of s*c (log2 units), possibly stale by < 8
-    float l = 0.0f;       // this half's running sum of bf16(2^(s*c - m)): normalises O
-    float lx = 0.0f;      // this half's running sum of 2^(s*c - m) in fp32: the log-sum-exp
+    const float2 c2 = make_float2(c, c);
+    float m0 = -INFINITY, m1 = -INFINITY;  // running row maxima of s*c (log2), may lag by < 8
+    float l0 = 0.0f, l1 = 0.0f;            // this thread's partial sums of bf16(2^(s*c - m))
+    float lx0 = 0.0f, lx1 = 0.0f;          // the same in fp32 (log-sum-exp)
     bool ok = true;
-    uint32_t xphase = 0;  // phases completed on this row pair's exchange barrier
 
     for (int j = 0; j < nkv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(t), static_cast<uint32_t>(j) & 1u, ctl));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t sr[2][32];
-      ptx::tmem_ld32(tS + half * 64, sr[0]);
-      ptx::tmem_ld32(tS + half * 64 + 32, sr[1]);
-      ptx::tmem_wait_ld();
-      float s[64];
+      // s0[e] / s1[e], e = 2k + i, is the score of key 8k + 2*cq + i for row r0 / r1
+      float s0[32], s1[32];
 #pragma unroll
-      for (int q = 0; q < 2; ++q)
+      for (int hb = 0; hb < 2; ++hb) {
+        uint32_t r[32];
+        ptx::tmem_ld_16x256b_x8(tS + hb * 64, r);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[q * 32 + i] = __uint_as_float(sr[q][i]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const int k = hb * 8 + kk;
+          s0[2 * k] = __uint_as_float(r[4 * kk]);
+          s0[2 * k + 1] = __uint_as_float(r[4 * kk + 1]);
+          s1[2 * k] = __uint_as_float(r[4 * kk + 2]);
+          s1[2 * k + 1] = __uint_as_float(r[4 * kk + 3]);
+        }
+      }
       if (j == nkv - 1 && kv_last_valid < kBN) {
-        const int lim = kv_last_valid - half * 64;  // keys of this half that exist
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= lim) s[i] = -INFINITY;
-      }
-      // this half's row max: four independent chains of three-input maxima
-      float ma = fmaxf(s[0], s[1]), mb = fmaxf(s[2], s[3]);
-      float mc = fmaxf(s[4], s[5]), md = fmaxf(s[6], s[7]);
-#pragma unroll
-      for (int i = 8; i < 64; i += 8) {
-        ma = ptx::max3(ma, s[i], s[i + 1]);
-        mb = ptx::max3(mb, s[i + 2], s[i + 3]);
-        mc = ptx::max3(mc, s[i + 4], s[i + 5]);
-        md = ptx::max3(md, s[i + 6], s[i + 7]);
-      }
-      // trade maxima with the other half of the row (buffers alternate by step parity)
-      const int par = (j & 1) * kParityStride;
-      xmine[par] = ptx::max3(ma, mb, fmaxf(mc, md));
-      ptx::mbar_arrive(xbar);
-      ok = __all_sync(0xffffffffu, mbar_wait(xbar, xphase & 1u, ctl));
-      ++xphase;
-      if (!ok) break;
-      const float mx = fmaxf(xmine[par], xpeer[par]);
-      const float cand = mx * c;
-      const bool grow = cand > m + kRescaleThreshold;  // identical in both halves
-      const float alpha = grow ? ptx::ex2_approx(m - cand) : 1.0f;
-      if (grow) m = cand;
-      l *= alpha;
-      if (kLse) lx *= alpha;
-      // P = 2^(s*c - m), rounded to bf16, written over S (this half: 32 packed columns)
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
-      float2 acc[2], accx[2];
-#pragma unroll
-      for (int k = 0; k < 2; ++k) acc[k] = accx[k] = make_float2(0.0f, 0.0f);
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float2 x = __ffma2_rn(make_float2(s[2 * i], s[2 * i + 1]), c2, nm2);
-        float2 pe;
-        if (kEmuEvery > 0 && (i % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
-          pe = exp2_poly2(x);
-        } else {
-          pe = make_float2(ptx::ex2_approx(x.x), ptx::ex2_approx(x.y));
-        }
-        pk[i] = ptx::pack_bf16x2(pe.x, pe.y);
-        acc[i & 1] = __fadd2_rn(acc[i & 1], make_float2(__uint_as_float(pk[i] << 16),
-                                                        __uint_as_float(pk[i] & 0xFFFF0000u)));
-        if (kLse) accx[i & 1] = __fadd2_rn(accx[i & 1], pe);
-      }
-      ptx::tmem_st32(tS + half * 32, pk);
-      {
-        const float2 a = __fadd2_rn(acc[0], acc[1]);
-        l += a.x + a.y;
-        if (kLse) {
-          const float2 b = __fadd2_rn(accx[0], accx[1]);
-          lx += b.x + b.y;
+        for (int e = 0; e < 32; ++e) {
+          const int key = 8 * (e >> 1) + 2 * cq + (e & 1);
+          if (key >= kv_last_valid) s0[e] = s1[e] = -INFINITY;
         }
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+      // row maxima: this thread's 32 keys, then the quad
+      float a0 = fmaxf(s0[0], s0[1]), b0 = fmaxf(s0[2], s0[3]);
+      float a1 = fmaxf(s1[0], s1[1]), b1 = fmaxf(s1[2], s1[3]);
+#pragma unroll
+      for (int e = 4; e < 32; e += 4) {
+        a0 = ptx::max3(a0, s0[e], s0[e + 1]);
+        b0 = ptx::max3(b0, s0[e + 2], s0[e + 3]);
+        a1 = ptx::max3(a1, s1[e], s1[e + 1]);
+        b1 = ptx::max3(b1, s1[e + 2], s1[e + 3]);
+      }
+      float mx0 = fmaxf(a0, b0), mx1 = fmaxf(a1, b1);
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float cand0 = mx0 * c, cand1 = mx1 * c;
+      const bool grow0 = cand0 > m0 + kRescaleThreshold;  // identical in the row's 4 threads
+      const bool grow1 = cand1 > m1 + kRescaleThreshold;
+      const float alpha0 = grow0 ? ptx::ex2_approx(m0 - cand0) : 1.0f;
+      const float alpha1 = grow1 ? ptx::ex2_approx(m1 - cand1) : 1.0f;
+      if (grow0) m0 = cand0;
+      if (grow1) m1 = cand1;
+      // P = 2^(s*c - m) rounded to bf16, stored over S as packed pairs: the pair of
+      // keys 8k + 2*cq + {0,1} is packed column 4k + cq (16x128b shape)
+      const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
+      float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+      float2 accx0 = make_float2(0.0f, 0.0f), accx1 = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int k = hb * 8 + kk;
+          const float2 x0 = __ffma2_rn(make_float2(s0[2 * k], s0[2 * k + 1]), c2, nm0);
+          const float2 x1 = __ffma2_rn(make_float2(s1[2 * k], s1[2 * k + 1]), c2, nm1);
+          float2 e0, e1;
+          if (kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+            e0 = exp2_poly2(x0);
+            e1 = exp2_poly2(x1);
+          } else {
+            e0 = make_float2(ptx::ex2_approx(x0.x), ptx::ex2_approx(x0.y));
+            e1 = make_float2(ptx::ex2_approx(x1.x), ptx::ex2_approx(x1.y));
+          }
+          pk[2 * kk] = ptx::pack_bf16x2(e0.x, e0.y);
+          pk[2 * kk + 1] = ptx::pack_bf16x2(e1.x, e1.y);
+          acc0 = __fadd2_rn(acc0, make_float2(__uint_as_float(pk[2 * kk] << 16),
+                                              __uint_as_float(pk[2 * kk] & 0xFFFF0000u)));
+          acc1 = __fadd2_rn(acc1, make_float2(__uint_as_float(pk[2 * kk + 1] << 16),
+                                              __uint_as_float(pk[2 * kk + 1] & 0xFFFF0000u)));
+          if (kLse) {
+            accx0 = __fadd2_rn(accx0, e0);
+            accx1 = __fadd2_rn(accx1, e1);
+          }
+        }
+        ptx::tmem_st_16x128b_x8(tS + hb * 32, pk);
+      }
+      l0 = l0 * alpha0 + (acc0.x + acc0.y);
+      l1 = l1 * alpha1 + (acc1.x + acc1.y);
+      if (kLse) {
+        lx0 = lx0 * alpha0 + (accx0.x + accx0.y);
+        lx1 = lx1 * alpha1 + (accx1.x + accx1.y);
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow0 || grow1)) {
         // O_t(j-1) is final once S_t(j) has landed (the tensor core runs in issue
-        // order); the explicit wait keeps that visible.  Rescale this half in place.
+        // order); the explicit wait keeps that visible.  Rescale it in place.
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(t), static_cast<uint32_t>(j - 1) & 1u, ctl));
         if (!ok) break;
         ptx::tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < D / 64; ++q) {
-          uint32_t orr[32];
-          ptx::tmem_ld32(tO + q * 32, orr);
+        for (int hb = 0; hb < D / 64; ++hb) {
+          uint32_t r[32];
+          ptx::tmem_ld_16x256b_x8(tO + hb * 64, r);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-          ptx::tmem_st32(tO + q * 32, orr);
+          for (int kk = 0; kk < 8; ++kk) {
+            r[4 * kk] = __float_as_uint(__uint_as_float(r[4 * kk]) * alpha0);
+            r[4 * kk + 1] = __float_as_uint(__uint_as_float(r[4 * kk + 1]) * alpha0);
+            r[4 * kk + 2] = __float_as_uint(__uint_as_float(r[4 * kk + 2]) * alpha1);
+            r[4 * kk + 3] = __float_as_uint(__uint_as_float(r[4 * kk + 3]) * alpha1);
+          }
+          ptx::tmem_st_16x256b_x8(tO + hb * 64, r);
         }
       }
       ptx::tmem_wait_st();
@@ -444,52 +507,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(t), static_cast<uint32_t>(nkv - 1) & 1u, ctl));
     }
     if (ok) {
-      // the two halves add their row sums (the buffer the last step did not use)
-      const int par = (nkv & 1) * kParityStride;
-      xmine[par] = l;
-      ptx::mbar_arrive(xbar);
-      ok = __all_sync(0xffffffffu, mbar_wait(xbar, xphase & 1u, ctl));
-      ++xphase;
-    }
-    if (ok) {
-      const int par = (nkv & 1) * kParityStride;
-      const float l_row = xmine[par] + xpeer[par];
+      // a row's sums: add the quad's partials
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
       ptx::tc_fence_after();
-      const int64_t row = q_row0 + t * kBM + row_in_tile;  // within the sequence
-      const bool valid = row < seq_len;
-      const float inv_l = 1.0f / l_row;
-      uint16_t* orow = p.o + static_cast<int64_t>(batch) * p.o_batch + (seq_base + row) * p.o_tok +
-                       static_cast<int64_t>(head) * p.o_head + half * (D / 2);
+      const int64_t row0 = q_row0 + t * kBM + r0, row1 = q_row0 + t * kBM + r1;  // within the sequence
+      const bool v0 = row0 < seq_len, v1 = row1 < seq_len;
+      const float inv0 = 1.0f / l0, inv1 = 1.0f / l1;
+      uint16_t* const obase = p.o + static_cast<int64_t>(batch) * p.o_batch + static_cast<int64_t>(head) * p.o_head;
+      uint32_t* const o0 = reinterpret_cast<uint32_t*>(obase + (seq_base + row0) * p.o_tok) + cq;
+      uint32_t* const o1 = reinterpret_cast<uint32_t*>(obase + (seq_base + row1) * p.o_tok) + cq;
 #pragma unroll
-      for (int q = 0; q < D / 64; ++q) {
-        uint32_t orr[32];
-        ptx::tmem_ld32(tO + q * 32, orr);
+      for (int hb = 0; hb < D / 64; ++hb) {
+        uint32_t r[32];
+        ptx::tmem_ld_16x256b_x8(tO + hb * 64, r);
         ptx::tmem_wait_ld();
-        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = ptx::pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const int k = hb * 8 + kk;  // columns 8k + 2*cq + {0,1}: the 32-bit word 4k + cq
+          if (v0) o0[4 * k] = ptx::pack_bf16x2(__uint_as_float(r[4 * kk]) * inv0, __uint_as_float(r[4 * kk + 1]) * inv0);
+          if (v1) o1[4 * k] = ptx::pack_bf16x2(__uint_as_float(r[4 * kk + 2]) * inv1, __uint_as_float(r[4 * kk + 3]) * inv1);
         }
       }
       if (kLse) {
-        // a second round for the unrounded sums, in the other buffer (whose last
-        // reader, the peer's final step, finished before the round above)
-        const int par2 = ((nkv + 1) & 1) * kParityStride;
-        xmine[par2] = lx;
-        ptx::mbar_arrive(xbar);
-        ok = __all_sync(0xffffffffu, mbar_wait(xbar, xphase & 1u, ctl));
-        ++xphase;
-        if (ok && half == 0 && valid) {
-          const float lx_row = xmine[par2] + xpeer[par2];
-          const float v = (m + log2f(lx_row)) * 0.69314718055994530942f;
+        lx0 += __shfl_xor_sync(0xffffffffu, lx0, 1);
+        lx1 += __shfl_xor_sync(0xffffffffu, lx1, 1);
+        lx0 += __shfl_xor_sync(0xffffffffu, lx0, 2);
+        lx1 += __shfl_xor_sync(0xffffffffu, lx1, 2);
+        if (cq == 0) {
+          const float ln2 = 0.69314718055994530942f;
           if (kVarlen) {
-            p.lse[static_cast<int64_t>(head) * p.total + seq_base + row] = v;
+            float* lrow = p.lse + static_cast<int64_t>(head) * p.total + seq_base;
+            if (v0) lrow[row0] = (m0 + log2f(lx0)) * ln2;
+            if (v1) lrow[row1] = (m1 + log2f(lx1)) * ln2;
           } else {
-            p.lse[(static_cast<int64_t>(batch) * p.n_heads + head) * p.seqlen + row] = v;
+            float* lrow = p.lse + (static_cast<int64_t>(batch) * p.n_heads + head) * p.seqlen;
+            if (v0) lrow[row0] = (m0 + log2f(lx0)) * ln2;
+            if (v1) lrow[row1] = (m1 + log2f(lx1)) * ln2;
           }
         }
       }
