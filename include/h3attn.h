@@ -12,7 +12,7 @@
  *     RMSNorm, RoPE and layout kernel is listed as missing; Implemented And
  *     Validated: "H3 packed denoising" (video and audio tokens in one
  *     sequence) and "Ragged Ulysses sequence parallelism" (ragged sequences).
- *   - "Buyer Questions Status", block composition answer: in the profiled
+ *   - "Buyer Questions: Current Evidence Status", block composition answer: in the profiled
  *     DiT block, attention is the largest share of time and norm/RoPE feeds it;
  *     strided-NHD Q/K/V (no copy of the QKV projection output) was a measured
  *     saving.
@@ -100,9 +100,10 @@ int h3attn_device_status(void* stream, int clear);
  *        (required when pos is given; values other than 0, 1, 2 act as 0).
  * sec_t + sec_h + sec_w must equal head_dim, each even (checked only when pos
  * is given).  head_dim: 64 or 128.  n_tokens == 0 is a no-op.
- * Arithmetic: sum of squares and scaling in fp32; the rotation in fp64 from
- * fp64 angles, so every output is within one bf16 ulp of the exactly rounded
- * result.
+ * Arithmetic: sum of squares and scaling in fp32; angles and their sine and
+ * cosine in fp64, each carried as a pair of floats (head + tail), and the
+ * rotation in fp32 with error-free products, so every output is within one
+ * bf16 ulp of the exactly rounded result.
  */
 h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, void* k_out,
                               int64_t n_tokens, int32_t n_heads, int32_t head_dim,

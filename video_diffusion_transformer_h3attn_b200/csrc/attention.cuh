@@ -54,6 +54,7 @@ constexpr int kAttnThreads = 640;
 // Registers: 640 threads launch at 96 per thread (five warps per scheduler x 96 <= 512);
 // a softmax thread holds 64 scores, so every role fits without a setmaxnreg split.
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+constexpr int kSortMax = 256;              // ragged batches up to this many sequences run longest first
 
 template <int D>
 struct AttnTraits {
@@ -64,7 +65,8 @@ struct AttnTraits {
   static constexpr int kTiles = kQTiles + kStages;
   // barriers: q, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2]
   static constexpr int kBarriers = 1 + 2 * kStages + 3 * kQTiles;
-  static constexpr int kSmemBytes = 1024 /*alignment slack*/ + kTiles * kTileBytes + 8 * kBarriers + 16;
+  static constexpr int kSmemBytes =
+      1024 /*alignment slack*/ + kTiles * kTileBytes + 8 * kBarriers + 16 + 8 * kSortMax;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(256 + kQTiles * D <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -144,20 +146,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto bar_o_done = [&](int t) { return bars + 8u * (1 + 2 * kS + 2 * kQTiles + t); };
   volatile uint32_t* const slot_words =
       reinterpret_cast<volatile uint32_t*>(base_ptr + T::kTiles * T::kTileBytes + 8 * T::kBarriers);
-  // slot_words[0] = tensor-memory base, [1] = work valid, [2] = sequence, [3] = query-pair index
+  // slot_words[0] = tensor-memory base, [1] = work valid, [2] = sequence, [3] = query-pair index,
+  // then the ragged scheduler's scratch (2 x kSortMax ints)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const LaunchCtl ctl = p.ctl;
 
   // ---- work decode (CTA-uniform, published through shared memory) ----------------
+  // Ragged batches: the query-tile pairs of all sequences are numbered longest
+  // sequence first (FLOPs grow with the square of the length, so the last CTAs of
+  // the launch are the cheapest); with more than kSortMax sequences, in given order.
+  int32_t* const sched = reinterpret_cast<int32_t*>(
+      const_cast<uint32_t*>(slot_words) + 4);  // [kSortMax] lengths, then [kSortMax] order
+  if (kVarlen && p.nseq <= kSortMax) {
+    const int n = p.nseq;
+    if (threadIdx.x < n) sched[threadIdx.x] = p.cu_seqlens[threadIdx.x + 1] - p.cu_seqlens[threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x < n) {
+      const int32_t mine = sched[threadIdx.x];
+      int rank = 0;
+      for (int i = 0; i < n; ++i) {
+        const int32_t other = sched[i];
+        rank += (other > mine || (other == mine && i < static_cast<int>(threadIdx.x))) ? 1 : 0;
+      }
+      sched[kSortMax + rank] = static_cast<int32_t>(threadIdx.x);
+    }
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
     uint32_t valid = launch_failed(ctl) ? 0u : 1u;
     uint32_t seq = 0, pair = blockIdx.x;
     if (kVarlen && valid) {
       valid = 0;
       uint32_t x = blockIdx.x;
-      for (int s = 0; s < p.nseq; ++s) {
+      const bool sorted = p.nseq <= kSortMax;
+      for (int i = 0; i < p.nseq; ++i) {
+        const int s = sorted ? sched[kSortMax + i] : i;
         const int32_t n = p.cu_seqlens[s + 1] - p.cu_seqlens[s];
         const uint32_t pairs = n > 0 ? static_cast<uint32_t>((n + kQTiles * kBM - 1) / (kQTiles * kBM)) : 0u;
         if (x < pairs) {
@@ -459,10 +484,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           pk[2 * kk] = ptx::pack_bf16x2(e0.x, e0.y);
           pk[2 * kk + 1] = ptx::pack_bf16x2(e1.x, e1.y);
-          acc0 = __fadd2_rn(acc0, make_float2(__uint_as_float(pk[2 * kk] << 16),
-                                              __uint_as_float(pk[2 * kk] & 0xFFFF0000u)));
-          acc1 = __fadd2_rn(acc1, make_float2(__uint_as_float(pk[2 * kk + 1] << 16),
-                                              __uint_as_float(pk[2 * kk + 1] & 0xFFFF0000u)));
+          ptx::add_bf16x2_f32(acc0.x, acc0.y, pk[2 * kk]);
+          ptx::add_bf16x2_f32(acc1.x, acc1.y, pk[2 * kk + 1]);
           if (kLse) {
             accx0 = __fadd2_rn(accx0, e0);
             accx1 = __fadd2_rn(accx1, e1);

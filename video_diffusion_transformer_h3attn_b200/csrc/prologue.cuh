@@ -15,9 +15,10 @@
 //
 // Precision: x*gamma is exact in fp32 (8-bit x 8-bit significands) and the
 // RMS scale factor r multiplies a whole row, so it only adds a relative error.
-// The rotation of (x*gamma) runs in fp64, which removes the absolute error of a
-// fp32 rotation when the two terms cancel.  The result is therefore within a
-// few fp32 ulps (relative) of the exact value, i.e. within one bf16 ulp of its
+// The rotation of (x*gamma) uses cos/sin computed in fp64 and carried as float
+// pairs, with error-free products, which removes the absolute error a plain fp32
+// rotation has when its two terms cancel.  The result is therefore within a few
+// fp32 ulps (relative) of the exact value, i.e. within one bf16 ulp of its
 // correctly rounded bf16.  The kernel is HBM-bound: two reads and two writes of
 // n_tokens * n_heads * d bf16 values.
 #pragma once
@@ -113,7 +114,10 @@ __global__ void __launch_bounds__(256) prologue_kernel(const __grid_constant__ P
     }
   }
   const bool do_rope = kind != 0;
-  double cs[4], sn[4];
+  // cos and sin as unevaluated float pairs (hi + lo, |lo| <= ulp(hi)/2): the
+  // rotation below then runs in fp32 with error-free products, avoiding per-element
+  // fp32 <-> fp64 conversions (which share the slow conversion pipe).
+  float ch[4], cl[4], sh[4], sl[4];
   if (do_rope) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -126,7 +130,12 @@ __global__ void __launch_bounds__(256) prologue_kernel(const __grid_constant__ P
       } else {
         angle = static_cast<double>(pt) * p.rope.inv_freq_1d[pair];
       }
-      sincos(angle, &sn[k], &cs[k]);
+      double sd, cd;
+      sincos(angle, &sd, &cd);
+      ch[k] = static_cast<float>(cd);
+      cl[k] = static_cast<float>(cd - static_cast<double>(ch[k]));
+      sh[k] = static_cast<float>(sd);
+      sl[k] = static_cast<float>(sd - static_cast<double>(sh[k]));
     }
   }
 
@@ -168,11 +177,20 @@ __global__ void __launch_bounds__(256) prologue_kernel(const __grid_constant__ P
       if (do_rope) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const double a0 = x[2 * k], a1 = x[2 * k + 1];
-          const double t0 = fma(a0, cs[k], -a1 * sn[k]);
-          const double t1 = fma(a0, sn[k], a1 * cs[k]);
-          y[2 * k] = static_cast<float>(t0) * r;
-          y[2 * k + 1] = static_cast<float>(t1) * r;
+          // (a0, a1) = x*gamma is exact in fp32.  Each product a*c_hi is split into
+          // its rounded value and exact error (fma), so the difference of the two
+          // large products is exact when they nearly cancel (Sterbenz) and the small
+          // terms carry the rest: the rotated value has a relative error of a few
+          // fp32 ulps even when its two terms cancel.
+          const float a0 = x[2 * k], a1 = x[2 * k + 1];
+          const float p0 = a0 * ch[k], e0 = fmaf(a0, ch[k], -p0);
+          const float q0 = a1 * sh[k], f0 = fmaf(a1, sh[k], -q0);
+          const float t0 = (p0 - q0) + (fmaf(a0, cl[k], e0) - fmaf(a1, sl[k], f0));
+          const float p1 = a0 * sh[k], e1 = fmaf(a0, sh[k], -p1);
+          const float q1 = a1 * ch[k], f1 = fmaf(a1, ch[k], -q1);
+          const float t1 = (p1 + q1) + (fmaf(a0, sl[k], e1) + fmaf(a1, cl[k], f1));
+          y[2 * k] = t0 * r;
+          y[2 * k + 1] = t1 * r;
         }
       } else {
 #pragma unroll

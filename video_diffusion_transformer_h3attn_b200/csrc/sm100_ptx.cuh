@@ -376,5 +376,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// lo += float(low bf16 of x), hi += float(high bf16 of x): sm_100 mixed-precision
+// add (the bf16 operand widens exactly, one fp32 rounding per add).
+__device__ __forceinline__ void add_bf16x2_f32(float& lo, float& hi, uint32_t x) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+      : "+f"(lo), "+f"(hi) : "r"(x));
+}
+
 }  // namespace ptx
 }  // namespace h3
