@@ -364,6 +364,7 @@ def run_gpu(args):
     flops = w.attention_flops()
     value = world * flops / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
+    merge_line = measure_merge(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
     att_tflops = flops / (att_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     pro_bytes = 4.0 * w.total * w.n_heads * w.head_dim * 2 + 12.0 * w.total + w.total + 4 * w.head_dim
@@ -395,6 +396,7 @@ def run_gpu(args):
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "overlap": "uploads and downloads on two copy streams under the previous/next step's kernels"},
+        "roofline_merge": merge_line,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(),
     }
@@ -411,6 +413,40 @@ def run_gpu(args):
     return 0
 
 
+def measure_merge(h3, w, dev, stream, steps, peaks, peak_src):
+    """The log-sum-exp merge of two partial results (a key-split schedule's
+    combine step) on the workload's full output shape, timed on its own after
+    the step measurements: HBM-bound, 3 rows of d bf16 + 3 fp32 per (token, head)."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(5)
+    shape = (1, w.total, w.n_heads, w.head_dim)
+    oa = torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    ob = torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    la = torch.randn((1, w.n_heads, w.total), generator=g, device=dev) * 4
+    lb = torch.randn((1, w.n_heads, w.total), generator=g, device=dev) * 4
+    o = torch.empty_like(oa)
+    lse = torch.empty_like(la)
+    for _ in range(3):
+        h3.merge(oa, la, ob, lb, o=o, lse=lse)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        h3.merge(oa, la, ob, lb, o=o, lse=lse)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h3.device_status()
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = 3.0 * w.total * w.n_heads * (w.head_dim * 2 + 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del oa, ob, la, lb, o, lse
+    return {"bound": "hbm", "achieved": gbs, "peak": peaks.get("hbm_gbs"), "unit": "GB/s",
+            "frac": gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "ms": ms,
+            "bytes_per_launch": nbytes, "kernel": "merge_kernel<128>", "peak_source": peak_src,
+            "note": "not part of the step: the combine of two partial results over split keys, "
+                    "on this workload's output shape"}
+
+
 def run_kernel_only(args):
     """W + K launches of one kernel on one workload and nothing else (for ncu captures)."""
     import torch
@@ -425,7 +461,17 @@ def run_kernel_only(args):
 
     q, k, v = bf16(w.q), bf16(w.k), bf16(w.v)
     out = torch.empty_like(q)
-    if args.kernel_only == "prologue":
+    if args.kernel_only == "merge":
+        g = torch.Generator(device="cuda").manual_seed(5)
+        shape = (1, w.total, w.n_heads, w.head_dim)
+        oa = torch.randn(shape, generator=g, device="cuda").to(torch.bfloat16)
+        ob = torch.randn(shape, generator=g, device="cuda").to(torch.bfloat16)
+        la = torch.randn((1, w.n_heads, w.total), generator=g, device="cuda")
+        lb = torch.randn((1, w.n_heads, w.total), generator=g, device="cuda")
+        lo = torch.empty_like(la)
+        run = lambda: h3.merge(oa, la, ob, lb, o=out.view(shape), lse=lo)
+        unit = 3.0 * w.total * w.n_heads * (w.head_dim * 2 + 4) / 1e9
+    elif args.kernel_only == "prologue":
         g = (bf16(w.gamma_q), bf16(w.gamma_k)) if w.gamma_q is not None else (None, None)
         pos = torch.from_numpy(w.pos).cuda() if w.pos is not None else None
         kind = torch.from_numpy(w.kind).cuda() if w.kind is not None else None
@@ -452,7 +498,7 @@ def run_kernel_only(args):
     ms = e0.elapsed_time(e1) / args.steps
     print(json.dumps({"kernel": args.kernel_only, "workload": args.workload, "ms": ms,
                       "rate": unit / (ms * 1e-3),
-                      "rate_unit": "GB/s" if args.kernel_only == "prologue" else "TFLOP/s"}), flush=True)
+                      "rate_unit": "TFLOP/s" if args.kernel_only == "attention" else "GB/s"}), flush=True)
     return 0
 
 
@@ -465,7 +511,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload for --kernel-only runs (tiny, small, joint, 2k, ragged)")
-    ap.add_argument("--kernel-only", choices=["attention", "prologue"],
+    ap.add_argument("--kernel-only", choices=["attention", "prologue", "merge"],
                     help="launch only this kernel W + K times (profiling runs)")
     args = ap.parse_args()
     if args.kernel_only:

@@ -154,6 +154,59 @@ h3attn_status h3attn_fwd_varlen(const void* q, const void* k, const void* v, voi
                                 const int64_t v_strides[2], const int64_t o_strides[2],
                                 float softmax_scale, float* lse, void* stream);
 
+/*
+ * Partial attention and its combination: the pieces of a key-split schedule.
+ *
+ * Sequence-parallel execution of the block ("H3 Runtime Current State",
+ * Implemented And Validated: ragged Ulysses sequence parallelism and
+ * sequence-sharded block execution) can also split the KEYS of a sequence
+ * across steps or ranks.  For the same query rows, each key block gives a
+ * partial result (O_p, LSE_p): O_p the softmax-weighted mean of the block's
+ * values, LSE_p the natural log of the block's total weight sum_j exp(s_j).
+ * Combining all blocks by their LSE gives exactly the attention over all keys,
+ * up to rounding.
+ */
+
+/*
+ * h3attn_fwd_kv -- h3attn_fwd with the key/value length separate from the query
+ * length: each of the seqlen_q query rows of a sequence attends to the
+ * seqlen_kv key/value rows of the same batch entry.
+ *
+ * q, o: bf16 [batch][seqlen_q][n_heads][head_dim];  k, v: bf16
+ *   [batch][seqlen_kv][n_heads][head_dim]; strides {batch, token, head}.
+ * seqlen_q >= 1.  seqlen_kv >= 0: with no keys the result is the empty sum,
+ *   O = 0 and LSE = -inf (k and v are not read and may be NULL).
+ * lse: NULL, or fp32 [batch][n_heads][seqlen_q].  Other rules as h3attn_fwd,
+ * which is this call with seqlen_kv = seqlen_q.
+ */
+h3attn_status h3attn_fwd_kv(const void* q, const void* k, const void* v, void* o, int32_t batch,
+                            int64_t seqlen_q, int64_t seqlen_kv, int32_t n_heads, int32_t head_dim,
+                            const int64_t q_strides[3], const int64_t k_strides[3],
+                            const int64_t v_strides[3], const int64_t o_strides[3],
+                            float softmax_scale, float* lse, void* stream);
+
+/*
+ * h3attn_merge -- combine two partial results of the same query rows over
+ * disjoint key sets:
+ *   L = log(exp(lse_a) + exp(lse_b))  (formed as M + log(sum exp(lse_p - M)),
+ *                                      M = max(lse_a, lse_b)),
+ *   O = exp(lse_a - L) * O_a + exp(lse_b - L) * O_b.
+ * A part with lse = -inf is empty and has no weight (its O values must still be
+ * finite, as h3attn_fwd_kv writes them); two empty parts give O = 0, L = -inf.
+ *
+ * o_a, o_b, o: bf16 [batch][seqlen][n_heads][head_dim], strides {batch, token,
+ *   head}.  lse_a, lse_b, lse: fp32 [batch][n_heads][seqlen], contiguous.
+ * In place is allowed: o == o_a (same strides) with lse == lse_a, or likewise
+ *   with the b part; other overlaps are not.
+ * Arithmetic: weights in fp32 (expf, logf), O = fma(w_a, O_a, w_b * O_b) in
+ *   fp32, rounded once to bf16.
+ * seqlen == 0 is a no-op.  Alignment rules as every call; head_dim 64 or 128.
+ */
+h3attn_status h3attn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b,
+                           void* o, float* lse, int32_t batch, int64_t seqlen, int32_t n_heads,
+                           int32_t head_dim, const int64_t oa_strides[3], const int64_t ob_strides[3],
+                           const int64_t o_strides[3], void* stream);
+
 #ifdef __cplusplus
 }
 #endif

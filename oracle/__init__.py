@@ -64,6 +64,10 @@ class Oracle:
                                          _I32, _I32, _I32, _D, _P, _P]
         lib.h3o_attention.restype = ctypes.c_int
         lib.h3o_attention.argtypes = [_P, _P, _P, _I64, _I32, _I32, _P, _I32, _D, _P, _I64, _P, _P]
+        lib.h3o_attention_kv.restype = ctypes.c_int
+        lib.h3o_attention_kv.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _D, _P, _P]
+        lib.h3o_merge.restype = ctypes.c_int
+        lib.h3o_merge.argtypes = [_P, _P, _I32, _I64, _I32, _P, _P]
         self.lib = lib
 
     # -- bfloat16 rounding --------------------------------------------------------
@@ -127,6 +131,53 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle attention rejected its arguments (%d)" % rc)
         return o, lse
+
+    def attention_kv(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_q=None, cu_k=None,
+                     scale: Optional[float] = None) -> Tuple[np.ndarray, np.ndarray]:
+        """Each segment's queries against that segment's rows of a separate key set.
+
+        q: bf16 bits [total_q, H, d]; k, v: [total_k, H, d]; cu_q / cu_k: segment
+        bounds (default: one segment each).  Returns (o [total_q, H, d], lse [total_q, H]);
+        an empty key range gives o = 0, lse = -inf."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        total_q, H, d = q.shape
+        k = np.ascontiguousarray(k, dtype=np.uint16).reshape(-1, H, d)
+        v = np.ascontiguousarray(v, dtype=np.uint16).reshape(-1, H, d)
+        total_k = k.shape[0]
+        cq = np.ascontiguousarray([0, total_q] if cu_q is None else cu_q, dtype=np.int32)
+        ck = np.ascontiguousarray([0, total_k] if cu_k is None else cu_k, dtype=np.int32)
+        if len(cq) != len(ck):
+            raise ValueError("cu_q and cu_k must have the same number of segments")
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        o = np.empty((total_q, H, d), dtype=np.float64)
+        lse = np.empty((total_q, H), dtype=np.float64)
+        rc = self.lib.h3o_attention_kv(_ptr(q), total_q, _ptr(k), _ptr(v), total_k, H, d, _ptr(cq),
+                                       _ptr(ck), len(cq) - 1, float(scale), _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle attention_kv rejected its arguments (%d)" % rc)
+        return o, lse
+
+    def merge(self, o_parts, lse_parts) -> Tuple[np.ndarray, np.ndarray]:
+        """Combine partial results over disjoint key sets by their log-sum-exp.
+
+        o_parts: [P, ..., d] (any float), lse_parts: [P, ...] matching o_parts[..., 0].
+        Returns (o [..., d], lse [...]) in float64."""
+        o_parts = np.asarray(o_parts, dtype=np.float64)
+        lse_parts = np.asarray(lse_parts, dtype=np.float64)
+        if o_parts.shape[:-1] != lse_parts.shape:
+            raise ValueError("o_parts [P, ..., d] and lse_parts [P, ...] disagree")
+        n_parts, d = o_parts.shape[0], o_parts.shape[-1]
+        rows_shape = o_parts.shape[1:-1]
+        n_rows = int(np.prod(rows_shape)) if rows_shape else 1
+        op = np.ascontiguousarray(o_parts.reshape(n_parts, n_rows, d))
+        lp = np.ascontiguousarray(lse_parts.reshape(n_parts, n_rows))
+        o = np.empty((n_rows, d), dtype=np.float64)
+        lse = np.empty(n_rows, dtype=np.float64)
+        rc = self.lib.h3o_merge(_ptr(op), _ptr(lp), n_parts, n_rows, d, _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle merge rejected its arguments (%d)" % rc)
+        return o.reshape(*rows_shape, d), lse.reshape(rows_shape)
 
     # -- composition: the whole hot path ------------------------------------------------
     def prologue_workload(self, w, want_f64: bool = False):

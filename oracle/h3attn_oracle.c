@@ -31,6 +31,13 @@
  *             lse = max_j s_j + log(sum_j p_j).
  *   Order:    RMSNorm, then RoPE, then one rounding to bfloat16 (nearest,
  *             ties to even) -- the interface tensor attention consumes.
+ *   Partials: attention of queries against one block of a split key set, and
+ *             the combination of such partial results by their log-sum-exp
+ *             (h3o_attention_kv, h3o_merge): the pieces a key-split schedule of
+ *             the sequence-parallel attention ("H3 Runtime Current State",
+ *             "Ragged Ulysses sequence parallelism", "Sequence-sharded 50-block
+ *             execution") needs; the identity that the combined parts equal the
+ *             attention over all keys is what pins them.
  *
  * Every loop below is the definition written out in double precision, in the
  * order stated, with no blocking, fusion or reordering.
@@ -214,5 +221,104 @@ int h3o_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64
     }
     free(kd);
     free(vd);
+    return 0;
+}
+
+/*
+ * Attention of each segment's query rows against a separate set of key/value
+ * rows: segment s's queries [cu_q[s], cu_q[s+1]) of q attend to the keys
+ * [cu_k[s], cu_k[s+1]) of k and v.  This is the partial attention a key-split
+ * (context-parallel) schedule computes per key block; its (o, lse) pairs are
+ * combined by h3o_merge.  The arithmetic is the definition above; an empty key
+ * range is an empty sum: o = 0 and lse = -inf.
+ *   q: bf16 bits [total_q][n_heads][d];  k, v: [total_k][n_heads][d].
+ *   o: double [total_q][n_heads][d];     lse: double [total_q][n_heads] or NULL.
+ * Returns 0, or -1 on invalid arguments.
+ */
+int h3o_attention_kv(const uint16_t* q, int64_t total_q, const uint16_t* k, const uint16_t* v,
+                     int64_t total_k, int32_t n_heads, int32_t d, const int32_t* cu_q,
+                     const int32_t* cu_k, int32_t nseq, double scale, double* o, double* lse) {
+    if (!q || !o || !cu_q || !cu_k || total_q < 0 || total_k < 0 || n_heads <= 0 || d <= 0 ||
+        d > 1024 || nseq <= 0)
+        return -1;
+    if (total_k > 0 && (!k || !v)) return -1;
+    if (cu_q[0] != 0 || cu_q[nseq] != total_q || cu_k[0] != 0 || cu_k[nseq] != total_k) return -1;
+    for (int s = 0; s < nseq; ++s)
+        if (cu_q[s + 1] < cu_q[s] || cu_k[s + 1] < cu_k[s]) return -1;
+    for (int h = 0; h < n_heads; ++h) {
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t t = 0; t < total_q; ++t) {
+            int seg = 0;
+            while (!(cu_q[seg] <= t && t < cu_q[seg + 1])) ++seg;
+            const int64_t kb = cu_k[seg], ke = cu_k[seg + 1];
+            double* row_o = o + (t * n_heads + h) * (int64_t)d;
+            if (ke == kb) {  /* no keys: the empty sum */
+                for (int i = 0; i < d; ++i) row_o[i] = 0.0;
+                if (lse) lse[t * n_heads + h] = -INFINITY;
+                continue;
+            }
+            double qv[1024];
+            for (int i = 0; i < d; ++i) qv[i] = h3o_bf16_to_double(q[(t * n_heads + h) * (int64_t)d + i]);
+            double* s_row = (double*)malloc(sizeof(double) * (size_t)(ke - kb));
+            double m = -INFINITY;
+            for (int64_t j = kb; j < ke; ++j) {
+                double qk = 0.0;
+                for (int i = 0; i < d; ++i) qk += qv[i] * h3o_bf16_to_double(k[(j * n_heads + h) * (int64_t)d + i]);
+                s_row[j - kb] = scale * qk;
+                if (s_row[j - kb] > m) m = s_row[j - kb];
+            }
+            double num[1024];
+            for (int i = 0; i < d; ++i) num[i] = 0.0;
+            double z = 0.0;
+            for (int64_t j = kb; j < ke; ++j) {
+                const double w = exp(s_row[j - kb] - m);
+                z += w;
+                for (int i = 0; i < d; ++i) num[i] += w * h3o_bf16_to_double(v[(j * n_heads + h) * (int64_t)d + i]);
+            }
+            for (int i = 0; i < d; ++i) row_o[i] = num[i] / z;
+            if (lse) lse[t * n_heads + h] = m + log(z);
+            free(s_row);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Combination of partial attention results over disjoint key sets, by their
+ * log-sum-exp: with L = log(sum_p exp(lse_p)), o = sum_p exp(lse_p - L) o_p.
+ * (Each o_p is its part's weighted mean of values with total weight exp(lse_p);
+ * the whole mean weights each part by its share of the total.)  L is formed as
+ * M + log(sum_p exp(lse_p - M)) with M = max_p lse_p.  Parts with lse = -inf
+ * are empty and carry no weight; a row whose parts are all empty gives o = 0,
+ * L = -inf.
+ *   o_parts:   double [n_parts][n_rows][d];  lse_parts: double [n_parts][n_rows].
+ *   o:         double [n_rows][d];           lse:       double [n_rows].
+ * Returns 0, or -1 on invalid arguments.
+ */
+int h3o_merge(const double* o_parts, const double* lse_parts, int32_t n_parts, int64_t n_rows,
+              int32_t d, double* o, double* lse) {
+    if (!o_parts || !lse_parts || !o || !lse || n_parts <= 0 || n_rows < 0 || d <= 0) return -1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r) {
+        double mx = -INFINITY;
+        for (int p = 0; p < n_parts; ++p)
+            if (lse_parts[p * n_rows + r] > mx) mx = lse_parts[p * n_rows + r];
+        double* out = o + r * d;
+        if (mx == -INFINITY) {
+            for (int i = 0; i < d; ++i) out[i] = 0.0;
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double den = 0.0;
+        for (int p = 0; p < n_parts; ++p) den += exp(lse_parts[p * n_rows + r] - mx);
+        const double L = mx + log(den);
+        for (int i = 0; i < d; ++i) out[i] = 0.0;
+        for (int p = 0; p < n_parts; ++p) {
+            const double w = exp(lse_parts[p * n_rows + r] - L);
+            const double* op = o_parts + (p * n_rows + r) * (int64_t)d;
+            for (int i = 0; i < d; ++i) out[i] += w * op[i];
+        }
+        lse[r] = L;
+    }
     return 0;
 }

@@ -380,6 +380,84 @@ def pin_attention_special_cases(orc):
     _close(lrows, lse[rows], 0, 0, "sampled rows (lse)")
 
 
+# ----------------------------------------------------------------------------------
+# partial attention over a split key set, and the log-sum-exp merge
+# ----------------------------------------------------------------------------------
+
+
+def pin_attention_kv_library(orc):
+    """Queries against a key set of another length: torch SDPA in float64."""
+    rng = np.random.default_rng(29)
+    Nq, Nk, H, d = 23, 41, 2, 16
+    q = to_bf16_bits_f32(rng.standard_normal((Nq, H, d)) * 1.5)
+    k = to_bf16_bits_f32(rng.standard_normal((Nk, H, d)))
+    v = to_bf16_bits_f32(rng.standard_normal((Nk, H, d)))
+    o, lse = orc.attention_kv(q, k, v)
+    qt, kt, vt = (torch.from_numpy(bf16_value(a)).permute(1, 0, 2) for a in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).permute(1, 0, 2).numpy()
+    _close(o, ref, 1e-12, 1e-14, "attention_kv vs torch sdpa float64")
+    sc = torch.einsum("hnd,hmd->hnm", qt, kt) / math.sqrt(d)
+    _close(lse, torch.logsumexp(sc, -1).T.numpy(), 1e-12, 1e-14, "attention_kv lse vs torch.logsumexp")
+    # segments: each segment's queries see only its own key rows; an empty key range is the empty sum
+    cu_q, cu_k = [0, 5, 5, 23], [0, 17, 30, 30]
+    os_, ls = orc.attention_kv(q, k[:30], v[:30], cu_q, cu_k)
+    o0, l0 = orc.attention_kv(q[:5], k[:17], v[:17])
+    _close(os_[:5], o0, 0, 0, "attention_kv segment 0")
+    _close(ls[:5], l0, 0, 0, "attention_kv segment 0 lse")
+    _close(os_[5:], np.zeros((18, H, d)), 0, 0, "empty key range gives o = 0")
+    assert np.all(np.isneginf(ls[5:])), "empty key range gives lse = -inf"
+    # the mpmath brute force of the self-attention pins applies with cu_q == cu_k
+    cu = np.array([0, 2, 6], dtype=np.int32)
+    qs = to_bf16_bits_f32(rng.standard_normal((6, 1, 8)))
+    ks = to_bf16_bits_f32(rng.standard_normal((6, 1, 8)))
+    vs = to_bf16_bits_f32(rng.standard_normal((6, 1, 8)))
+    ob, lb = orc.attention_kv(qs, ks, vs, cu, cu, scale=0.61)
+    wo, wl = _mp_attention(qs, ks, vs, cu, 0.61)
+    _close(ob, wo, 1e-13, 1e-15, "attention_kv vs mpmath (o)")
+    _close(lb, wl, 1e-13, 1e-15, "attention_kv vs mpmath (lse)")
+
+
+def pin_merge(orc):
+    """Merging the parts of a split key set gives the attention over all keys."""
+    rng = np.random.default_rng(31)
+    Nq, Nk, H, d = 19, 64, 3, 16
+    q = to_bf16_bits_f32(rng.standard_normal((Nq, H, d)) * 2)
+    k = to_bf16_bits_f32(rng.standard_normal((Nk, H, d)))
+    v = to_bf16_bits_f32(rng.standard_normal((Nk, H, d)))
+    full_o, full_l = orc.attention_kv(q, k, v)
+    for cuts in ([0, 30, 64], [0, 1, 2, 50, 64], [0, 0, 64], [0, 64, 64]):
+        parts = [orc.attention_kv(q, k[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+        o, l = orc.merge(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+        _close(o, full_o, 1e-13, 1e-15, "merge of %s equals the whole (o)" % cuts)
+        _close(l, full_l, 1e-13, 1e-15, "merge of %s equals the whole (lse)" % cuts)
+    # closed forms on synthetic parts
+    a = rng.standard_normal((5, 8))
+    b = rng.standard_normal((5, 8))
+    la = rng.standard_normal(5)
+    o, l = orc.merge(a[None], la[None])
+    _close(o, a, 0, 0, "one part is itself")
+    _close(l, la, 0, 0, "one part keeps its lse")
+    o, l = orc.merge(np.stack([a, b]), np.stack([la, la]))
+    _close(o, (a + b) / 2, 1e-15, 1e-15, "equal weights average")
+    _close(l, la + math.log(2), 1e-15, 1e-15, "equal weights add log 2")
+    lb = la + math.log(3)  # b carries three times a's weight
+    o, l = orc.merge(np.stack([a, b]), np.stack([la, lb]))
+    _close(o, (a + 3 * b) / 4, 1e-14, 1e-15, "weights 1:3")
+    _close(l, la + math.log(4), 1e-14, 1e-15, "lse of weights 1:3")
+    o2, l2 = orc.merge(np.stack([b, a]), np.stack([lb, la]))
+    _close(o2, o, 1e-15, 0, "order of parts")
+    ninf = np.full(5, -np.inf)
+    o, l = orc.merge(np.stack([a, b]), np.stack([la, ninf]))
+    _close(o, a, 1e-15, 0, "an empty part carries no weight")
+    o, l = orc.merge(np.stack([a, b]), np.stack([ninf, ninf]))
+    _close(o, np.zeros_like(a), 0, 0, "all parts empty gives o = 0")
+    assert np.all(np.isneginf(l)), "all parts empty gives lse = -inf"
+    # large lse values: the max shift keeps it finite (the inputs la + 900 are only
+    # good to ulp(900) ~ 1.1e-13, which bounds the agreement)
+    o, l = orc.merge(np.stack([a, b]), np.stack([la + 900.0, la + 900.0 + math.log(3)]))
+    _close(o, (a + 3 * b) / 4, 1e-12, 1e-12, "weights 1:3 at lse ~ 900")
+
+
 ALL_PINS = [
     pin_bf16_rounding,
     pin_rmsnorm,
@@ -389,4 +467,6 @@ ALL_PINS = [
     pin_attention_brute_force,
     pin_attention_library,
     pin_attention_special_cases,
+    pin_attention_kv_library,
+    pin_merge,
 ]

@@ -20,7 +20,8 @@ def lib():
 def test_exports_every_declared_symbol(lib):
     names = h3.declared_symbols()
     assert set(names) >= {"h3attn_prologue", "h3attn_fwd", "h3attn_fwd_varlen", "h3attn_version",
-                          "h3attn_status_string", "h3attn_last_error", "h3attn_device_status"}
+                          "h3attn_status_string", "h3attn_last_error", "h3attn_device_status",
+                          "h3attn_fwd_kv", "h3attn_merge"}
     for n in names:
         assert hasattr(lib, n), "library does not export %s" % n
 
@@ -72,6 +73,38 @@ def test_varlen_rejects_bad_arguments(lib):
     assert varlen(lib, max_seqlen=301) == INVALID
     assert varlen(lib, d=80) == UNSUPPORTED
     assert varlen(lib, strides=(257, 128)) == MISALIGNED
+
+
+def fwd_kv(lib, Nq=256, Nk=100, d=128, strides=(256 * 256, 256, 128), k=FAKE):
+    s = S3(*strides)
+    return lib.h3attn_fwd_kv(FAKE, k, FAKE, FAKE, 1, Nq, Nk, 2, d, s, s, s, s, 0.0, None, None)
+
+
+def test_fwd_kv_rejects_bad_arguments(lib):
+    assert fwd_kv(lib, Nq=0) == INVALID
+    assert fwd_kv(lib, Nk=-1) == INVALID
+    assert fwd_kv(lib, k=None) == INVALID
+    assert fwd_kv(lib, k=FAKE + 2) == MISALIGNED
+    assert fwd_kv(lib, d=32) == UNSUPPORTED
+    assert fwd_kv(lib, Nk=(1 << 30) + 1) == UNSUPPORTED
+    assert fwd_kv(lib, strides=(256 * 256, 252, 128)) == MISALIGNED
+
+
+def merge(lib, N=100, d=128, la=FAKE, o=FAKE, strides=(256 * 100, 256, 128), H=2):
+    s = S3(*strides)
+    return lib.h3attn_merge(FAKE, la, FAKE, FAKE, o, FAKE, 1, N, H, d, s, s, s, None)
+
+
+def test_merge_rejects_bad_arguments(lib):
+    assert merge(lib, la=None) == INVALID
+    assert merge(lib, o=None) == INVALID
+    assert merge(lib, N=-1) == INVALID
+    assert merge(lib, H=0) == INVALID
+    assert merge(lib, d=96) == UNSUPPORTED
+    assert merge(lib, la=FAKE + 2) == MISALIGNED
+    assert merge(lib, o=FAKE + 4) == MISALIGNED
+    assert merge(lib, strides=(256 * 100, 260, 128)) == MISALIGNED
+    assert merge(lib, N=0) == OK  # nothing to do: validated, nothing enqueued
 
 
 def prologue(lib, n=10, H=2, d=128, gq=FAKE, pos=FAKE, kind=FAKE, sec=(32, 48, 48), eps=1e-6,

@@ -29,6 +29,13 @@ MUTANTS = {
     "attn_no_max_shift": ("double p = exp(sc[j - j0] - mx);", "double p = exp(sc[j - j0]);"),
     "attn_boundary": ("t < cu_seqlens[s + 1])) ++s;", "t <= cu_seqlens[s + 1])) ++s;"),
     "attn_no_normalise": ("out[i] = acc[i] / den;", "out[i] = acc[i];"),
+    "kv_scale_dropped": ("s_row[j - kb] = scale * qk;", "s_row[j - kb] = qk;"),
+    "kv_lse_no_max": ("lse[t * n_heads + h] = m + log(z);", "lse[t * n_heads + h] = log(z);"),
+    "kv_segment_keys": ("const int64_t kb = cu_k[seg], ke = cu_k[seg + 1];",
+                        "const int64_t kb = cu_q[seg], ke = cu_q[seg + 1];"),
+    "merge_weight_unnormalised": ("const double w = exp(lse_parts[p * n_rows + r] - L);",
+                                  "const double w = exp(lse_parts[p * n_rows + r] - mx);"),
+    "merge_lse_is_max": ("const double L = mx + log(den);", "const double L = mx;"),
     "bf16_round_half_up": ("nearbyint(ax / quantum)", "floor(ax / quantum + 0.5)"),
     "bf16_subnormal_quantum": ("quantum = ldexp(1.0, -133);", "quantum = ldexp(1.0, -134);"),
     "bf16_mantissa_bits": ("quantum = ldexp(1.0, e - 1 - 7);", "quantum = ldexp(1.0, e - 1 - 8);"),

@@ -1,0 +1,81 @@
+"""The GPU side of Ulysses sequence parallelism on one GPU.
+
+The multi-rank exchange itself is covered on CPU ranks (tests/test_ulysses.py).
+Here the CUDA kernels are checked for the two properties that make the P-rank
+output equal the one-rank output bit for bit:
+  * the prologue applied to one head group of a shard (a strided view) and
+    written into that group's send block gives the same bits as the prologue of
+    the whole tensor, sliced;
+  * attention over a subset of the heads gives the same bits as those heads of
+    the attention over all heads;
+and the one-rank path of ulysses_attention equals the direct calls."""
+import numpy as np
+import pytest
+
+from h3_testlib import to_cuda_bf16
+from video_diffusion_transformer_h3attn_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h3():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import video_diffusion_transformer_h3attn_b200 as mod
+    return mod
+
+
+def _joint_like(n_video_grid=(4, 12, 16), n_audio=40, H=24, d=128, seed=41):
+    pos, kind = inputs.video_layout(*n_video_grid, n_audio=n_audio)
+    return inputs.make_workload("ulysses_gpu", [len(kind)], H, d, seed, pos=pos, kind=kind)
+
+
+@pytest.mark.parametrize("world", [2, 3, 4, 8])
+def test_prologue_into_head_group_blocks(h3, world):
+    import torch
+    w = _joint_like()
+    q, k = to_cuda_bf16(w.q), to_cuda_bf16(w.k)
+    g = (to_cuda_bf16(w.gamma_q), to_cuda_bf16(w.gamma_k))
+    pos, kind = torch.from_numpy(w.pos).cuda(), torch.from_numpy(w.kind).cuda()
+    full_q, full_k = h3.prologue(q, k, gamma_q=g[0], gamma_k=g[1], pos=pos, kind=kind)
+    n, H, d = q.shape
+    Hp = H // world
+    send_q = torch.empty((world, n, Hp, d), dtype=q.dtype, device=q.device)
+    send_k = torch.empty_like(send_q)
+    for p in range(world):
+        hs = slice(p * Hp, (p + 1) * Hp)
+        h3.prologue(q[:, hs], k[:, hs], send_q[p], send_k[p], g[0], g[1], pos=pos, kind=kind)
+    h3.device_status()
+    for p in range(world):
+        hs = slice(p * Hp, (p + 1) * Hp)
+        assert torch.equal(send_q[p], full_q[:, hs]) and torch.equal(send_k[p], full_k[:, hs])
+
+
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_head_subset_attention_is_bitwise_identical(h3, world):
+    import torch
+    w = inputs.random_case([3000], 24, 128, seed=43)
+    q, k, v = to_cuda_bf16(w.q), to_cuda_bf16(w.k), to_cuda_bf16(w.v)
+    full = h3.attention(q, k, v)
+    Hp = 24 // world
+    for p in range(world):
+        hs = slice(p * Hp, (p + 1) * Hp)
+        part = h3.attention(q[:, hs].contiguous(), k[:, hs].contiguous(), v[:, hs].contiguous())
+        assert torch.equal(part, full[:, hs]), "head group %d differs" % p
+    h3.device_status()
+
+
+def test_ulysses_one_rank_equals_direct_calls(h3):
+    import torch
+    from video_diffusion_transformer_h3attn_b200 import ulysses
+    w = _joint_like()
+    q, k, v = to_cuda_bf16(w.q), to_cuda_bf16(w.k), to_cuda_bf16(w.v)
+    g = (to_cuda_bf16(w.gamma_q), to_cuda_bf16(w.gamma_k))
+    pos, kind = torch.from_numpy(w.pos).cuda(), torch.from_numpy(w.kind).cuda()
+    o = ulysses.ulysses_attention(q, k, v, [q.shape[0]], gamma_q=g[0], gamma_k=g[1], pos=pos, kind=kind)
+    qp, kp = h3.prologue(q, k, gamma_q=g[0], gamma_k=g[1], pos=pos, kind=kind)
+    ref = h3.attention(qp, kp, v)
+    h3.device_status()
+    assert torch.equal(o, ref)

@@ -68,6 +68,12 @@ def library() -> ctypes.CDLL:
         lib.h3attn_fwd_varlen.restype = ctypes.c_int
         lib.h3attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I32, _I64_2,
                                           _I64_2, _I64_2, _I64_2, ctypes.c_float, _P, _P]
+        lib.h3attn_fwd_kv.restype = ctypes.c_int
+        lib.h3attn_fwd_kv.argtypes = [_P, _P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64_3, _I64_3,
+                                      _I64_3, _I64_3, ctypes.c_float, _P, _P]
+        lib.h3attn_merge.restype = ctypes.c_int
+        lib.h3attn_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I64_3, _I64_3,
+                                     _I64_3, _P]
         _lib = lib
     return _lib
 
@@ -215,3 +221,85 @@ def attention_varlen(q, k, v, cu_seqlens, max_seqlen: int, o=None,
         int(max_seqlen), H, d, st(q), st(k), st(v), st(o), float(softmax_scale or 0.0), _ptr(lse),
         _stream_handle(stream)))
     return (o, lse) if return_lse else o
+
+
+def _strides3(t):
+    """{batch, token, head} strides; a dimension of extent <= 1 is never stepped
+    over, so its stride (which torch may report as 0) is passed as a valid value."""
+    s = [t.stride(0), t.stride(1), t.stride(2)]
+    for i in range(3):
+        if t.shape[i] <= 1 and (s[i] <= 0 or s[i] % 8):
+            s[i] = 8
+    return _I64_3(*s)
+
+
+def attention_kv(q, k, v, o=None, softmax_scale: Optional[float] = None, return_lse: bool = False,
+                 stream=None):
+    """Queries against a key/value set of its own length (one block of a split key set).
+
+    q: bf16 CUDA [B, Nq, H, d] or [Nq, H, d]; k, v: [B, Nk, H, d] or [Nk, H, d], Nk >= 0.
+    Returns o (layout of q) and, with return_lse, lse fp32 [B, H, Nq]; Nk = 0 gives
+    o = 0 and lse = -inf."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16_cuda(name, t)
+    squeeze = q.dim() == 3
+    if squeeze:
+        q, k, v = q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0)
+        if o is not None:
+            o = o.unsqueeze(0)
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q must be [B, Nq, H, d] and k, v one [B, Nk, H, d] shape")
+    B, Nq, H, d = q.shape
+    if k.shape[0] != B or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k, v must match q in batch, heads and head_dim")
+    Nk = k.shape[1]
+    if o is None:
+        o = torch.empty((B, Nq, H, d), dtype=q.dtype, device=q.device)
+    _require_bf16_cuda("o", o)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if return_lse else None
+    st = _strides3
+    _check("h3attn_fwd_kv", library().h3attn_fwd_kv(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Nq, Nk, H, d, st(q), st(k), st(v), st(o),
+        float(softmax_scale or 0.0), _ptr(lse), _stream_handle(stream)))
+    out = o.squeeze(0) if squeeze else o
+    if return_lse:
+        return out, (lse.squeeze(0) if squeeze else lse)
+    return out
+
+
+def merge(o_a, lse_a, o_b, lse_b, o=None, lse=None, stream=None):
+    """Combine two partial results of the same queries over disjoint key sets.
+
+    o_a, o_b: bf16 CUDA [B, N, H, d] or [N, H, d]; lse_a, lse_b: fp32 CUDA [B, H, N]
+    or [H, N] (contiguous).  Returns (o, lse); o = o_a and lse = lse_a (or the b
+    pair) merge in place."""
+    torch = _torch()
+    for name, t in (("o_a", o_a), ("o_b", o_b)):
+        _require_bf16_cuda(name, t)
+    squeeze = o_a.dim() == 3
+    if squeeze:
+        o_a, o_b = o_a.unsqueeze(0), o_b.unsqueeze(0)
+        lse_a, lse_b = lse_a.unsqueeze(0), lse_b.unsqueeze(0)
+        o = None if o is None else o.unsqueeze(0)
+        lse = None if lse is None else lse.unsqueeze(0)
+    if o_a.dim() != 4 or o_b.shape != o_a.shape:
+        raise ValueError("o_a and o_b must share a [B, N, H, d] shape")
+    B, N, H, d = o_a.shape
+    for name, t in (("lse_a", lse_a), ("lse_b", lse_b)):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N):
+            raise TypeError("%s must be a contiguous CUDA float32 [B, H, N] tensor" % name)
+    if o is None:
+        o = torch.empty((B, N, H, d), dtype=o_a.dtype, device=o_a.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=o_a.device)
+    _require_bf16_cuda("o", o)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, N):
+        raise TypeError("lse must be a contiguous float32 [B, H, N] tensor")
+    st = _strides3
+    _check("h3attn_merge", library().h3attn_merge(
+        _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o), _ptr(lse), B, N, H, d,
+        st(o_a), st(o_b), st(o), _stream_handle(stream)))
+    if squeeze:
+        return o.squeeze(0), lse.squeeze(0)
+    return o, lse

@@ -22,7 +22,10 @@
 //     128 scores sit in four threads of one warp (32 each): row maxima and sums
 //     are two shuffles away, and two warps per scheduler work on each tile.  The
 //     running max m (log2 units) may lag the true max by < 8, so P <= 256 and O
-//     is rescaled in tensor memory only when the max grows by more;
+//     is rescaled in tensor memory only when the max grows by more.  The first
+//     half of P is computed with m as it stands while the tile's maxima are
+//     formed, and redone only when m must grow, so the max is off the step's
+//     critical path;
 //     p = 2^(s*c - m) with c = scale*log2(e), rounded to bf16 and stored over S
 //     with the 16x128b shape; l sums the rounded weights the PV product uses
 //     (they normalise to exactly one), lx the unrounded ones (log-sum-exp);
@@ -79,7 +82,8 @@ struct AttnParams {
   const int32_t* cu_seqlens;  // ragged only
   int32_t nseq;               // ragged only
   int32_t n_heads;
-  int64_t seqlen;             // dense: tokens per sequence
+  int64_t seqlen;             // dense: query tokens per sequence
+  int64_t seqlen_kv;          // dense: key/value tokens per sequence (may differ, may be 0)
   int64_t total;              // ragged: total tokens (LSE row stride per head)
   float scale_log2;           // softmax_scale * log2(e)
   LaunchCtl ctl;
@@ -214,8 +218,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     seq_len = p.seqlen;
   }
   const int64_t q_row0 = static_cast<int64_t>(slot_words[3]) * (kQTiles * kBM);
-  const int nkv = static_cast<int>((seq_len + kBN - 1) / kBN);
-  const int kv_last_valid = static_cast<int>(seq_len - static_cast<int64_t>(nkv - 1) * kBN);
+  const int64_t kv_len = kVarlen ? seq_len : p.seqlen_kv;  // keys this sequence's queries see
+  const int nkv = static_cast<int>((kv_len + kBN - 1) / kBN);
+  const int kv_last_valid = static_cast<int>(kv_len - static_cast<int64_t>(nkv - 1) * kBN);
+  if (nkv == 0) {
+    // no keys (a block of a split key set may be empty): the empty sum, O = 0 and
+    // LSE = -inf, for the CTA's rows; nothing else runs
+    const int64_t row = q_row0 + threadIdx.x;
+    if (threadIdx.x < kQTiles * kBM && row < seq_len) {
+      uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<int64_t>(batch) * p.o_batch +
+                                             (seq_base + row) * p.o_tok + static_cast<int64_t>(head) * p.o_head);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+      if (kLse) {
+        float* lrow = kVarlen ? p.lse + static_cast<int64_t>(head) * p.total + seq_base
+                              : p.lse + (static_cast<int64_t>(batch) * p.n_heads + head) * p.seqlen;
+        lrow[row] = -INFINITY;
+      }
+    }
+    return;
+  }
 
   // ---- setup: barriers and tensor memory --------------------------------------------
   if (warp == kLoadWarp && lane == 0) {
@@ -439,6 +461,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (key >= kv_last_valid) s0[e] = s1[e] = -INFINITY;
         }
       }
+      // P = 2^(s*c - m) rounded to bf16, stored over S as packed pairs: the pair of
+      // keys 8k + 2*cq + {0,1} is packed column 4k + cq (16x128b shape).
+      float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+      float2 accx0 = make_float2(0.0f, 0.0f), accx1 = make_float2(0.0f, 0.0f);
+      // one pair of keys (pair index k) for both rows: exponentials, packing, sums
+      auto p_pair = [&](float sa0, float sa1, float sb0, float sb1, float2 nm0, float2 nm1, int k,
+                        uint32_t& pa, uint32_t& pb) {
+        const float2 x0 = __ffma2_rn(make_float2(sa0, sa1), c2, nm0);
+        const float2 x1 = __ffma2_rn(make_float2(sb0, sb1), c2, nm1);
+        float2 e0, e1;
+        if (kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
+          e0 = exp2_poly2(x0);
+          e1 = exp2_poly2(x1);
+        } else {
+          e0 = make_float2(ptx::ex2_approx(x0.x), ptx::ex2_approx(x0.y));
+          e1 = make_float2(ptx::ex2_approx(x1.x), ptx::ex2_approx(x1.y));
+        }
+        pa = ptx::pack_bf16x2(e0.x, e0.y);
+        pb = ptx::pack_bf16x2(e1.x, e1.y);
+        ptx::add_bf16x2_f32(acc0.x, acc0.y, pa);
+        ptx::add_bf16x2_f32(acc1.x, acc1.y, pb);
+        if (kLse) {
+          accx0 = __fadd2_rn(accx0, e0);
+          accx1 = __fadd2_rn(accx1, e1);
+        }
+      };
+      uint32_t pk[16];
+      // First half (keys 0..63) with the running max m as it stands, while this
+      // tile's row maxima are formed beside it on another pipe.  Only where a max
+      // grows by more than the threshold (always at j = 0, rarely later) are m and
+      // that half redone, so the max is off the critical path of the step.
+      {
+        const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, k, pk[2 * k], pk[2 * k + 1]);
+      }
       // row maxima: this thread's 32 keys, then the quad
       float a0 = fmaxf(s0[0], s0[1]), b0 = fmaxf(s0[2], s0[3]);
       float a1 = fmaxf(s1[0], s1[1]), b1 = fmaxf(s1[2], s1[3]);
@@ -457,49 +516,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float cand0 = mx0 * c, cand1 = mx1 * c;
       const bool grow0 = cand0 > m0 + kRescaleThreshold;  // identical in the row's 4 threads
       const bool grow1 = cand1 > m1 + kRescaleThreshold;
-      const float alpha0 = grow0 ? ptx::ex2_approx(m0 - cand0) : 1.0f;
-      const float alpha1 = grow1 ? ptx::ex2_approx(m1 - cand1) : 1.0f;
-      if (grow0) m0 = cand0;
-      if (grow1) m1 = cand1;
-      // P = 2^(s*c - m) rounded to bf16, stored over S as packed pairs: the pair of
-      // keys 8k + 2*cq + {0,1} is packed column 4k + cq (16x128b shape)
-      const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
-      float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
-      float2 accx0 = make_float2(0.0f, 0.0f), accx1 = make_float2(0.0f, 0.0f);
+      float alpha0 = 1.0f, alpha1 = 1.0f;
+      const bool any_grow = __any_sync(0xffffffffu, grow0 || grow1);
+      if (any_grow) {
+        if (grow0) {
+          alpha0 = ptx::ex2_approx(m0 - cand0);
+          m0 = cand0;
+        }
+        if (grow1) {
+          alpha1 = ptx::ex2_approx(m1 - cand1);
+          m1 = cand1;
+        }
+        // redo the first half from the scores still in tensor memory (P has not
+        // been stored over them yet), 32 columns at a time to spare registers
+        acc0 = acc1 = accx0 = accx1 = make_float2(0.0f, 0.0f);
+        const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        uint32_t pk[16];
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t r[16];
+          ptx::tmem_ld_16x256b_x4(tS + ch * 32, r);
+          ptx::tmem_wait_ld();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int k = hb * 8 + kk;
-          const float2 x0 = __ffma2_rn(make_float2(s0[2 * k], s0[2 * k + 1]), c2, nm0);
-          const float2 x1 = __ffma2_rn(make_float2(s1[2 * k], s1[2 * k + 1]), c2, nm1);
-          float2 e0, e1;
-          if (kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
-            e0 = exp2_poly2(x0);
-            e1 = exp2_poly2(x1);
-          } else {
-            e0 = make_float2(ptx::ex2_approx(x0.x), ptx::ex2_approx(x0.y));
-            e1 = make_float2(ptx::ex2_approx(x1.x), ptx::ex2_approx(x1.y));
-          }
-          pk[2 * kk] = ptx::pack_bf16x2(e0.x, e0.y);
-          pk[2 * kk + 1] = ptx::pack_bf16x2(e1.x, e1.y);
-          ptx::add_bf16x2_f32(acc0.x, acc0.y, pk[2 * kk]);
-          ptx::add_bf16x2_f32(acc1.x, acc1.y, pk[2 * kk + 1]);
-          if (kLse) {
-            accx0 = __fadd2_rn(accx0, e0);
-            accx1 = __fadd2_rn(accx1, e1);
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = ch * 4 + kk;
+            float v[4] = {__uint_as_float(r[4 * kk]), __uint_as_float(r[4 * kk + 1]),
+                          __uint_as_float(r[4 * kk + 2]), __uint_as_float(r[4 * kk + 3])};
+            if (j == nkv - 1) {
+#pragma unroll
+              for (int i = 0; i < 2; ++i)
+                if (8 * k + 2 * cq + i >= kv_last_valid) v[i] = v[2 + i] = -INFINITY;
+            }
+            p_pair(v[0], v[1], v[2], v[3], nm0, nm1, k, pk[2 * k], pk[2 * k + 1]);
           }
         }
-        ptx::tmem_st_16x128b_x8(tS + hb * 32, pk);
       }
+      ptx::tmem_st_16x128b_x8(tS, pk);
+      // second half (keys 64..127) with the final m
+      {
+        const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int k = 8 + kk;
+          p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, k, pk[2 * kk], pk[2 * kk + 1]);
+        }
+      }
+      ptx::tmem_st_16x128b_x8(tS + 32, pk);
       l0 = l0 * alpha0 + (acc0.x + acc0.y);
       l1 = l1 * alpha1 + (acc1.x + acc1.y);
       if (kLse) {
         lx0 = lx0 * alpha0 + (accx0.x + accx0.y);
         lx1 = lx1 * alpha1 + (accx1.x + accx1.y);
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow0 || grow1)) {
+      if (j > 0 && any_grow) {
         // O_t(j-1) is final once S_t(j) has landed (the tensor core runs in issue
         // order); the explicit wait keeps that visible.  Rescale it in place.
         ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(t), static_cast<uint32_t>(j - 1) & 1u, ctl));

@@ -17,6 +17,7 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "merge.cuh"
 #include "prologue.cuh"
 
 namespace {
@@ -244,15 +245,21 @@ h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, v
   return H3ATTN_OK;
 }
 
-h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, int32_t batch,
-                         int64_t seqlen, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
-                         const int64_t k_strides[3], const int64_t v_strides[3],
-                         const int64_t o_strides[3], float softmax_scale, float* lse, void* stream) {
-  h3attn_status st = check_common(q, k, v, o, n_heads, head_dim);
+h3attn_status h3attn_fwd_kv(const void* q, const void* k, const void* v, void* o, int32_t batch,
+                            int64_t seqlen_q, int64_t seqlen_kv, int32_t n_heads, int32_t head_dim,
+                            const int64_t q_strides[3], const int64_t k_strides[3],
+                            const int64_t v_strides[3], const int64_t o_strides[3], float softmax_scale,
+                            float* lse, void* stream) {
+  if (seqlen_kv < 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen_kv must not be negative");
+  // with no keys, k and v are never read and may be null (an empty tensor's data pointer)
+  const void* k_chk = (seqlen_kv == 0 && !k) ? q : k;
+  const void* v_chk = (seqlen_kv == 0 && !v) ? q : v;
+  h3attn_status st = check_common(q, k_chk, v_chk, o, n_heads, head_dim);
   if (st != H3ATTN_OK) return st;
   if (batch <= 0 || batch > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "batch must be in [1, 65535]");
-  if (seqlen <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be positive");
-  if (seqlen > (int64_t(1) << 30)) return fail(H3ATTN_ERR_UNSUPPORTED, "seqlen too large");
+  if (seqlen_q <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be positive");
+  if (seqlen_q > (int64_t(1) << 30) || seqlen_kv > (int64_t(1) << 30))
+    return fail(H3ATTN_ERR_UNSUPPORTED, "seqlen too large");
   if ((st = check_strides(q_strides, 3, "q")) != H3ATTN_OK) return st;
   if ((st = check_strides(k_strides, 3, "k")) != H3ATTN_OK) return st;
   if ((st = check_strides(v_strides, 3, "v")) != H3ATTN_OK) return st;
@@ -261,9 +268,14 @@ h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, i
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(H3ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
 
   CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, head_dim, seqlen, n_heads, batch, q_strides[1], q_strides[2], q_strides[0])) != H3ATTN_OK) return st;
-  if ((st = make_map(&mk, k, head_dim, seqlen, n_heads, batch, k_strides[1], k_strides[2], k_strides[0])) != H3ATTN_OK) return st;
-  if ((st = make_map(&mv, v, head_dim, seqlen, n_heads, batch, v_strides[1], v_strides[2], v_strides[0])) != H3ATTN_OK) return st;
+  if ((st = make_map(&mq, q, head_dim, seqlen_q, n_heads, batch, q_strides[1], q_strides[2], q_strides[0])) != H3ATTN_OK) return st;
+  if (seqlen_kv > 0) {
+    if ((st = make_map(&mk, k, head_dim, seqlen_kv, n_heads, batch, k_strides[1], k_strides[2], k_strides[0])) != H3ATTN_OK) return st;
+    if ((st = make_map(&mv, v, head_dim, seqlen_kv, n_heads, batch, v_strides[1], v_strides[2], v_strides[0])) != H3ATTN_OK) return st;
+  } else {
+    mk = mq;  // no keys: the kernel writes the empty result and reads neither map
+    mv = mq;
+  }
 
   h3::AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
@@ -273,16 +285,71 @@ h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, i
   prm.o_head = o_strides[2];
   prm.lse = lse;
   prm.n_heads = n_heads;
-  prm.seqlen = seqlen;
-  prm.total = seqlen;
+  prm.seqlen = seqlen_q;
+  prm.seqlen_kv = seqlen_kv;
+  prm.total = seqlen_q;
   prm.scale_log2 = resolve_scale(softmax_scale, head_dim);
   prm.ctl.launch_id = next_launch_id();
 
-  const int64_t pairs = (seqlen + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM);
+  const int64_t pairs = (seqlen_q + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM);
   dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return head_dim == 128 ? launch_attention<128, false>(mq, mk, mv, prm, grid, s)
                          : launch_attention<64, false>(mq, mk, mv, prm, grid, s);
+}
+
+h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, int32_t batch,
+                         int64_t seqlen, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
+                         const int64_t k_strides[3], const int64_t v_strides[3],
+                         const int64_t o_strides[3], float softmax_scale, float* lse, void* stream) {
+  if (seqlen <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be positive");
+  return h3attn_fwd_kv(q, k, v, o, batch, seqlen, seqlen, n_heads, head_dim, q_strides, k_strides, v_strides,
+                       o_strides, softmax_scale, lse, stream);
+}
+
+h3attn_status h3attn_merge(const void* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o,
+                           float* lse, int32_t batch, int64_t seqlen, int32_t n_heads, int32_t head_dim,
+                           const int64_t oa_strides[3], const int64_t ob_strides[3],
+                           const int64_t o_strides[3], void* stream) {
+  if (!o_a || !o_b || !o || !lse_a || !lse_b || !lse) return fail(H3ATTN_ERR_INVALID_ARG, "null pointer");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(H3ATTN_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (batch <= 0 || batch > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "batch must be in [1, 65535]");
+  if (n_heads <= 0 || n_heads > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "n_heads must be in [1, 65535]");
+  if (seqlen < 0 || seqlen > (int64_t(1) << 30)) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be in [0, 2^30]");
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o))
+    return fail(H3ATTN_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(lse_a) | reinterpret_cast<uintptr_t>(lse_b) | reinterpret_cast<uintptr_t>(lse)) & 3u)
+    return fail(H3ATTN_ERR_MISALIGNED, "lse arrays must be 4-byte aligned");
+  h3attn_status st;
+  if ((st = check_strides(oa_strides, 3, "o_a")) != H3ATTN_OK) return st;
+  if ((st = check_strides(ob_strides, 3, "o_b")) != H3ATTN_OK) return st;
+  if ((st = check_strides(o_strides, 3, "o")) != H3ATTN_OK) return st;
+  if (seqlen == 0) return H3ATTN_OK;
+
+  h3::MergeParams prm;
+  prm.oa = static_cast<const uint16_t*>(o_a);
+  prm.ob = static_cast<const uint16_t*>(o_b);
+  prm.o = static_cast<uint16_t*>(o);
+  prm.oa_batch = oa_strides[0]; prm.oa_tok = oa_strides[1]; prm.oa_head = oa_strides[2];
+  prm.ob_batch = ob_strides[0]; prm.ob_tok = ob_strides[1]; prm.ob_head = ob_strides[2];
+  prm.o_batch = o_strides[0]; prm.o_tok = o_strides[1]; prm.o_head = o_strides[2];
+  prm.lse_a = lse_a;
+  prm.lse_b = lse_b;
+  prm.lse = lse;
+  prm.seqlen = seqlen;
+  prm.n_heads = n_heads;
+  dim3 grid(static_cast<unsigned>((seqlen + h3::kMergeTokens - 1) / h3::kMergeTokens),
+            static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 128) {
+    h3::merge_kernel<128><<<grid, h3::kMergeThreads, 0, s>>>(prm);
+  } else {
+    h3::merge_kernel<64><<<grid, h3::kMergeThreads, 0, s>>>(prm);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return H3ATTN_OK;
 }
 
 h3attn_status h3attn_fwd_varlen(const void* q, const void* k, const void* v, void* o,
