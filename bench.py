@@ -204,9 +204,14 @@ def run_reference(args):
 # -----------------------------------------------------------------------------------------
 # GPU arm
 # -----------------------------------------------------------------------------------------
+ATTENTION_SOURCES = ("attention.cuh", "sm100_ptx.cuh", "common.cuh")
+
+
 def source_hash():
+    """Hash of the attention kernel's sources (a stored ncu figure is only used
+    while these are unchanged)."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "video_diffusion_transformer_h3attn_b200", "csrc"))):
+    for f in ATTENTION_SOURCES:
         with open(os.path.join(ROOT, "video_diffusion_transformer_h3attn_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -365,6 +370,7 @@ def run_gpu(args):
     value = world * flops / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
     merge_line = measure_merge(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
+    qkv_line = measure_qkv(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
     att_tflops = flops / (att_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     pro_bytes = 4.0 * w.total * w.n_heads * w.head_dim * 2 + 12.0 * w.total + w.total + 4 * w.head_dim
@@ -397,6 +403,7 @@ def run_gpu(args):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "overlap": "uploads and downloads on two copy streams under the previous/next step's kernels"},
         "roofline_merge": merge_line,
+        "roofline_qkv": qkv_line,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(),
     }
@@ -447,6 +454,73 @@ def measure_merge(h3, w, dev, stream, steps, peaks, peak_src):
                     "on this workload's output shape"}
 
 
+def _qkv_inputs(w, dev):
+    """Token activations and a projection weight of the workload's model width
+    (dim_in = H*d, 3*H*d features), seeded; positions and gammas from the workload."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(7)
+    hd = w.n_heads * w.head_dim
+    x = torch.randn((w.total, hd), generator=g, device=dev).to(torch.bfloat16)
+    wt = (torch.randn((3 * hd, hd), generator=g, device=dev) / hd ** 0.5).to(torch.bfloat16)
+    bias = (torch.randn(3 * hd, generator=g, device=dev) * 0.1).to(torch.bfloat16)
+    return x, wt, bias
+
+
+def measure_qkv(h3, w, dev, stream, steps, peaks, peak_src):
+    """The Q/K/V projection with the prologue fused into its epilogue, on the
+    workload's token count at model width, against the unfused path (cuBLAS
+    projection, then the prologue kernel) timed the same way.  Not part of the step."""
+    import torch
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, wt, bias = _qkv_inputs(w, dev)
+    gq, gk = bf16(w.gamma_q), bf16(w.gamma_k)
+    pos, kind = torch.from_numpy(w.pos).to(dev), torch.from_numpy(w.kind).to(dev)
+    H, d = w.n_heads, w.head_dim
+    out = torch.empty((w.total, 3, H, d), dtype=torch.bfloat16, device=dev)
+    q, k, v = out[:, 0], out[:, 1], out[:, 2]
+
+    def fused():
+        h3.qkv_fused(x, wt, H, bias=bias, q_out=q, k_out=k, v_out=v, gamma_q=gq, gamma_k=gk, eps=w.eps,
+                     pos=pos, kind=kind, sections=w.sections, theta=w.theta)
+
+    proj = torch.empty((w.total, 3 * H * d), dtype=torch.bfloat16, device=dev)
+    qp = torch.empty((w.total, H, d), dtype=torch.bfloat16, device=dev)
+    kp = torch.empty_like(qp)
+
+    def unfused():
+        torch.addmm(bias, x, wt.T, out=proj)
+        pv = proj.view(w.total, 3, H, d)
+        h3.prologue(pv[:, 0], pv[:, 1], qp, kp, gq, gk, w.eps, pos, kind, w.sections, w.theta)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    ms = timed(fused)
+    h3.device_status()
+    ms_unfused = timed(unfused)
+    flops = 2.0 * w.total * (H * d) * (3 * H * d)
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    del x, wt, bias, out, proj, qp, kp
+    return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak, "ms": ms,
+            "unfused_ms": ms_unfused, "speedup_vs_unfused": ms_unfused / ms, "flops_per_launch": flops,
+            "kernel": "qkv_fused_kernel<%d>" % d, "peak_source": "%s bf16_tflops (kernel timed alone)" % peak_src,
+            "note": "not part of the step: projection dim_in = H*d to 3*H*d features with RMSNorm + RoPE in the "
+                    "epilogue, on this workload's tokens; unfused = cuBLAS addmm then the prologue kernel"}
+
+
 def run_kernel_only(args):
     """W + K launches of one kernel on one workload and nothing else (for ncu captures)."""
     import torch
@@ -461,7 +535,14 @@ def run_kernel_only(args):
 
     q, k, v = bf16(w.q), bf16(w.k), bf16(w.v)
     out = torch.empty_like(q)
-    if args.kernel_only == "merge":
+    if args.kernel_only == "qkv":
+        x, wt, bias = _qkv_inputs(w, "cuda")
+        gq, gk = bf16(w.gamma_q), bf16(w.gamma_k)
+        pos, kind = torch.from_numpy(w.pos).cuda(), torch.from_numpy(w.kind).cuda()
+        run = lambda: h3.qkv_fused(x, wt, w.n_heads, bias=bias, gamma_q=gq, gamma_k=gk, eps=w.eps, pos=pos,
+                                   kind=kind, sections=w.sections, theta=w.theta)
+        unit = 2.0 * w.total * (w.n_heads * w.head_dim) * (3 * w.n_heads * w.head_dim) / 1e12
+    elif args.kernel_only == "merge":
         g = torch.Generator(device="cuda").manual_seed(5)
         shape = (1, w.total, w.n_heads, w.head_dim)
         oa = torch.randn(shape, generator=g, device="cuda").to(torch.bfloat16)
@@ -498,7 +579,7 @@ def run_kernel_only(args):
     ms = e0.elapsed_time(e1) / args.steps
     print(json.dumps({"kernel": args.kernel_only, "workload": args.workload, "ms": ms,
                       "rate": unit / (ms * 1e-3),
-                      "rate_unit": "TFLOP/s" if args.kernel_only == "attention" else "GB/s"}), flush=True)
+                      "rate_unit": "TFLOP/s" if args.kernel_only in ("attention", "qkv") else "GB/s"}), flush=True)
     return 0
 
 
@@ -511,7 +592,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload for --kernel-only runs (tiny, small, joint, 2k, ragged)")
-    ap.add_argument("--kernel-only", choices=["attention", "prologue", "merge"],
+    ap.add_argument("--kernel-only", choices=["attention", "prologue", "merge", "qkv"],
                     help="launch only this kernel W + K times (profiling runs)")
     args = ap.parse_args()
     if args.kernel_only:

@@ -207,6 +207,43 @@ h3attn_status h3attn_merge(const void* o_a, const float* lse_a, const void* o_b,
                            int32_t head_dim, const int64_t oa_strides[3], const int64_t ob_strides[3],
                            const int64_t o_strides[3], void* stream);
 
+/*
+ * h3attn_qkv_fused -- the block's Q/K/V projection with the prologue fused into
+ * it: Q', K', V straight from the token activations.
+ *
+ * "H3 Runtime Current State", Owned Performance Kernels, lists fused Q/K
+ * RMSNorm, RoPE and layout work as missing; "Buyer Questions: Current Evidence
+ * Status" (block composition) has the projection feed norm/RoPE, with its
+ * strided NHD output read in place.  For token n and output feature
+ *   f = sum_c x[n][c] * w[f][c] (+ bias[f]),   f in [0, 3*n_heads*head_dim):
+ * features [0, H*d) are Q (head f / d), [H*d, 2*H*d) K, [2*H*d, 3*H*d) V.  Each
+ * (token, head) row of Q and of K then goes through RMSNorm (gamma_q / gamma_k;
+ * skipped where NULL) and RoPE (pos/kind/sections/theta exactly as
+ * h3attn_prologue; skipped where pos is NULL); V is the projection.  Every
+ * output is rounded once to bf16: the projection is not rounded before the norm.
+ *
+ * x:     bf16 [n_tokens][dim_in], token stride x_tok_stride (elements).
+ * w:     bf16 [3*n_heads*head_dim][dim_in], contiguous (the layout of a linear
+ *        layer's weight: one row per output feature).
+ * bias:  bf16 [3*n_heads*head_dim] or NULL.
+ * q_out, k_out, v_out: bf16 NHD outputs, strides {out_tok_strides[i],
+ *        out_head_strides[i]} for i = 0 (Q), 1 (K), 2 (V) -- three views of one
+ *        fused buffer work as they are.
+ * gamma_q, gamma_k: bf16 [head_dim] or NULL.  eps: inside the square root.
+ * pos, kind, sec_*, theta: as h3attn_prologue.
+ * Requirements: head_dim 64 or 128; n_heads*head_dim a multiple of 256;
+ *   dim_in a positive multiple of 64; n_tokens >= 0 (0 is a no-op).
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation; bias, sum of
+ *   squares, 1/rms (rsqrtf) and the gamma scale in fp32; RoPE with fp64 angles
+ *   whose cosine and sine are carried as float pairs and error-free products.
+ */
+h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, void* q_out, void* k_out,
+                               void* v_out, int64_t n_tokens, int32_t dim_in, int32_t n_heads,
+                               int32_t head_dim, int64_t x_tok_stride, const int64_t out_tok_strides[3],
+                               const int64_t out_head_strides[3], const void* gamma_q, const void* gamma_k,
+                               double eps, const int32_t* pos, const uint8_t* kind, int32_t sec_t,
+                               int32_t sec_h, int32_t sec_w, double theta, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,9 @@ class Oracle:
         lib.h3o_attention.argtypes = [_P, _P, _P, _I64, _I32, _I32, _P, _I32, _D, _P, _I64, _P, _P]
         lib.h3o_attention_kv.restype = ctypes.c_int
         lib.h3o_attention_kv.argtypes = [_P, _I64, _P, _P, _I64, _I32, _I32, _P, _P, _I32, _D, _P, _P]
+        lib.h3o_qkv_norm_rope.restype = ctypes.c_int
+        lib.h3o_qkv_norm_rope.argtypes = [_P, _I64, _I32, _I64, _P, _P, _I32, _I32, _P, _P, _D, _P, _P,
+                                          _I32, _I32, _I32, _D, _P, _I64, _P, _P, _P, _P, _P, _P]
         lib.h3o_merge.restype = ctypes.c_int
         lib.h3o_merge.argtypes = [_P, _P, _I32, _I64, _I32, _P, _P]
         self.lib = lib
@@ -178,6 +181,39 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle merge rejected its arguments (%d)" % rc)
         return o.reshape(*rows_shape, d), lse.reshape(rows_shape)
+
+    def qkv_norm_rope(self, x: np.ndarray, w: np.ndarray, bias: Optional[np.ndarray] = None,
+                      n_heads: int = 1, gamma_q=None, gamma_k=None, eps: float = 1e-6, pos=None,
+                      kind=None, sections=(32, 48, 48), theta: float = 10000.0,
+                      rows: Optional[np.ndarray] = None, want_f64: bool = True, want_bf16: bool = True):
+        """Q/K/V projection x w^T (+ bias), then RMSNorm + RoPE of Q and K per head.
+
+        x: bf16 bits [n_tokens, dim_in]; w: [3*H*d, dim_in]; bias: [3*H*d] or None.
+        Returns ((q64, k64, v64), (q16, k16, v16)), each [nrows, H, d] (None where not
+        wanted)."""
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w = np.ascontiguousarray(w, dtype=np.uint16)
+        n, dim_in = x.shape
+        H = int(n_heads)
+        d = w.shape[0] // (3 * H)
+        if w.shape != (3 * H * d, dim_in):
+            raise ValueError("w must be [3*H*d, dim_in]")
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+        gq = None if gamma_q is None else np.ascontiguousarray(gamma_q, dtype=np.uint16)
+        gk = None if gamma_k is None else np.ascontiguousarray(gamma_k, dtype=np.uint16)
+        p = None if pos is None else np.ascontiguousarray(pos, dtype=np.int32)
+        kd = None if kind is None else np.ascontiguousarray(kind, dtype=np.uint8)
+        r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+        nrows = n if r is None else len(r)
+        o64 = [np.empty((nrows, H, d)) if want_f64 else None for _ in range(3)]
+        o16 = [np.empty((nrows, H, d), dtype=np.uint16) if want_bf16 else None for _ in range(3)]
+        st, sh, sw = sections
+        rc = self.lib.h3o_qkv_norm_rope(_ptr(x), n, dim_in, dim_in, _ptr(w), _ptr(b), H, d, _ptr(gq),
+                                        _ptr(gk), float(eps), _ptr(p), _ptr(kd), st, sh, sw, float(theta),
+                                        _ptr(r), nrows, *(_ptr(a) for a in o64), *(_ptr(a) for a in o16))
+        if rc != 0:
+            raise ValueError("oracle qkv_norm_rope rejected its arguments (%d)" % rc)
+        return tuple(o64), tuple(o16)
 
     # -- composition: the whole hot path ------------------------------------------------
     def prologue_workload(self, w, want_f64: bool = False):

@@ -322,3 +322,76 @@ int h3o_merge(const double* o_parts, const double* lse_parts, int32_t n_parts, i
     }
     return 0;
 }
+
+/*
+ * The Q/K/V projection of the block followed by the per-head RMSNorm + RoPE of
+ * Q and K: the prologue fused into the projection that produces its input
+ * ("H3 Runtime Current State", Owned Performance Kernels: fused Q/K RMSNorm,
+ * RoPE and layout work; "Buyer Questions: Current Evidence Status", block
+ * composition: the projection output feeds norm/RoPE, and its strided NHD
+ * layout is read in place).  The projection is not rounded before the norm:
+ * the definition is the exact composition, rounded once at the end.
+ *   x:     bf16 bits, token n's row at x + n*s_x, dim_in values.
+ *   w:     bf16 bits [3*n_heads*d][dim_in] (one row per output feature).
+ *   bias:  bf16 bits [3*n_heads*d] or NULL.
+ *   Feature f = sum_c x[n][c] * w[f][c] (+ bias[f]); features [0, H*d) are Q
+ *   (head f / d), [H*d, 2*H*d) K, [2*H*d, 3*H*d) V.  Q and K rows of length d go
+ *   through RMSNorm (gamma_q / gamma_k when given, eps inside the root) and RoPE
+ *   (when pos is given) exactly as h3o_rmsnorm_rope; V is the projection.
+ *   rows:  int64 [nrows] token indices (NULL = every token).
+ *   q64, k64, v64: double [nrows][n_heads][d] or NULL (unrounded);
+ *   q16, k16, v16: bf16 bits, the same rounded once (NULL to skip).
+ * Returns 0, or -1 on invalid arguments.
+ */
+int h3o_qkv_norm_rope(const uint16_t* x, int64_t n_tokens, int32_t dim_in, int64_t s_x,
+                      const uint16_t* w, const uint16_t* bias, int32_t n_heads, int32_t d,
+                      const uint16_t* gamma_q, const uint16_t* gamma_k, double eps,
+                      const int32_t* pos, const uint8_t* kind, int32_t sec_t, int32_t sec_h,
+                      int32_t sec_w, double theta, const int64_t* rows, int64_t nrows,
+                      double* q64, double* k64, double* v64, uint16_t* q16, uint16_t* k16,
+                      uint16_t* v16) {
+    if (!x || !w || n_tokens < 0 || dim_in <= 0 || dim_in > 8192 || n_heads <= 0 || d <= 0 ||
+        d > 1024 || (d & 1))
+        return -1;
+    if (pos && (!kind || sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t & 1) || (sec_h & 1) ||
+                (sec_w & 1) || sec_t + sec_h + sec_w != d))
+        return -1;
+    if (!rows) nrows = n_tokens;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        if (t < 0 || t >= n_tokens) return -1;
+    }
+    const int64_t hd = (int64_t)n_heads * d;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t n = rows ? rows[r] : r;
+        double xin[8192];
+        for (int c = 0; c < dim_in; ++c) xin[c] = h3o_bf16_to_double(x[n * s_x + c]);
+        for (int part = 0; part < 3; ++part) {   /* 0 = Q, 1 = K, 2 = V */
+            const uint16_t* g = part == 0 ? gamma_q : part == 1 ? gamma_k : NULL;
+            double* out64 = part == 0 ? q64 : part == 1 ? k64 : v64;
+            uint16_t* out16 = part == 0 ? q16 : part == 1 ? k16 : v16;
+            for (int h = 0; h < n_heads; ++h) {
+                double feat[1024];
+                for (int i = 0; i < d; ++i) {
+                    const int64_t f = part * hd + (int64_t)h * d + i;
+                    double acc = 0.0;
+                    for (int c = 0; c < dim_in; ++c) acc += xin[c] * h3o_bf16_to_double(w[f * dim_in + c]);
+                    feat[i] = bias ? acc + h3o_bf16_to_double(bias[f]) : acc;
+                }
+                if (part < 2 && g) {
+                    double sq = 0.0;
+                    for (int i = 0; i < d; ++i) sq += feat[i] * feat[i];
+                    const double rms = sqrt(sq / (double)d + eps);
+                    for (int i = 0; i < d; ++i) feat[i] = feat[i] / rms * h3o_bf16_to_double(g[i]);
+                }
+                if (part < 2 && pos && kind[n] != 0)
+                    rope_row(feat, d, kind[n], pos + 3 * n, sec_t, sec_h, sec_w, theta);
+                const int64_t o = (r * n_heads + h) * (int64_t)d;
+                if (out64) for (int i = 0; i < d; ++i) out64[o + i] = feat[i];
+                if (out16) for (int i = 0; i < d; ++i) out16[o + i] = h3o_bf16_from_double(feat[i]);
+            }
+        }
+    }
+    return 0;
+}

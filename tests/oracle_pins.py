@@ -458,6 +458,50 @@ def pin_merge(orc):
     _close(o, (a + 3 * b) / 4, 1e-12, 1e-12, "weights 1:3 at lse ~ 900")
 
 
+# ----------------------------------------------------------------------------------
+# Q/K/V projection fused with the prologue
+# ----------------------------------------------------------------------------------
+
+
+def pin_qkv_projection(orc):
+    """The projection against numpy's float64 matmul; with identity weights the fused
+    operation is the pinned prologue itself."""
+    rng = np.random.default_rng(37)
+    n, H, d = 21, 2, 16
+    dim_in = 40
+    x = to_bf16_bits_f32(rng.standard_normal((n, dim_in)))
+    w = to_bf16_bits_f32(rng.standard_normal((3 * H * d, dim_in)) * 0.2)
+    b = to_bf16_bits_f32(rng.standard_normal(3 * H * d))
+    (q, k, v), _ = orc.qkv_norm_rope(x, w, b, n_heads=H, want_bf16=False)
+    ref = bf16_value(x) @ bf16_value(w).T + bf16_value(b)
+    _close(q.reshape(n, -1), ref[:, :H * d], 1e-13, 1e-13, "Q projection vs numpy")
+    _close(k.reshape(n, -1), ref[:, H * d:2 * H * d], 1e-13, 1e-13, "K projection vs numpy")
+    _close(v.reshape(n, -1), ref[:, 2 * H * d:], 1e-13, 1e-13, "V projection vs numpy")
+    # identity weights: Q, K, V are x itself, so norm + RoPE equal the prologue of x
+    sec = (4, 6, 6)
+    x2 = to_bf16_bits_f32(rng.standard_normal((n, H * d)))
+    eye = np.eye(H * d)
+    wi = to_bf16_bits_f32(np.concatenate([eye, eye, eye], axis=0))
+    gq = to_bf16_bits_f32(rng.uniform(0.5, 1.5, d))
+    gk = to_bf16_bits_f32(rng.uniform(0.5, 1.5, d))
+    pos = rng.integers(0, 20, size=(n, 3)).astype(np.int32)
+    kind = (np.arange(n) % 3).astype(np.uint8)
+    (q, k, v), (q16, _, v16) = orc.qkv_norm_rope(x2, wi, None, n_heads=H, gamma_q=gq, gamma_k=gk, pos=pos,
+                                                 kind=kind, sections=sec)
+    xh = x2.reshape(n, H, d)
+    rq, rq16 = orc.rmsnorm_rope(xh, gq, 1e-6, pos, kind, sec)
+    rk, _ = orc.rmsnorm_rope(xh, gk, 1e-6, pos, kind, sec)
+    _close(q, rq, 1e-15, 1e-15, "identity weights: Q = prologue(x)")
+    _close(k, rk, 1e-15, 1e-15, "identity weights: K = prologue(x) with gamma_k")
+    assert np.array_equal(q16, rq16), "identity weights: rounded Q = rounded prologue"
+    assert np.array_equal(v16, xh), "identity weights: V = x"
+    # sampled rows are the full computation's rows
+    rows = np.array([20, 0, 7], dtype=np.int64)
+    (qs, _, _), _ = orc.qkv_norm_rope(x2, wi, None, n_heads=H, gamma_q=gq, gamma_k=gk, pos=pos, kind=kind,
+                                      sections=sec, rows=rows)
+    _close(qs, q[rows], 0, 0, "sampled rows")
+
+
 ALL_PINS = [
     pin_bf16_rounding,
     pin_rmsnorm,
@@ -469,4 +513,5 @@ ALL_PINS = [
     pin_attention_special_cases,
     pin_attention_kv_library,
     pin_merge,
+    pin_qkv_projection,
 ]

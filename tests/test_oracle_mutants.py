@@ -36,6 +36,12 @@ MUTANTS = {
     "merge_weight_unnormalised": ("const double w = exp(lse_parts[p * n_rows + r] - L);",
                                   "const double w = exp(lse_parts[p * n_rows + r] - mx);"),
     "merge_lse_is_max": ("const double L = mx + log(den);", "const double L = mx;"),
+    "qkv_weight_transposed": ("acc += xin[c] * h3o_bf16_to_double(w[f * dim_in + c]);",
+                              "acc += xin[c] * h3o_bf16_to_double(w[c * dim_in + f % dim_in]);"),
+    "qkv_bias_dropped": ("feat[i] = bias ? acc + h3o_bf16_to_double(bias[f]) : acc;", "feat[i] = acc;"),
+    "qkv_k_uses_gamma_q": ("part == 1 ? gamma_k : NULL;", "part == 1 ? gamma_q : NULL;"),
+    "qkv_part_offset": ("const int64_t f = part * hd + (int64_t)h * d + i;",
+                        "const int64_t f = part * hd + (int64_t)h * d + (i ^ 1);"),
     "bf16_round_half_up": ("nearbyint(ax / quantum)", "floor(ax / quantum + 0.5)"),
     "bf16_subnormal_quantum": ("quantum = ldexp(1.0, -133);", "quantum = ldexp(1.0, -134);"),
     "bf16_mantissa_bits": ("quantum = ldexp(1.0, e - 1 - 7);", "quantum = ldexp(1.0, e - 1 - 8);"),

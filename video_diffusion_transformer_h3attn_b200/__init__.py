@@ -71,6 +71,9 @@ def library() -> ctypes.CDLL:
         lib.h3attn_fwd_kv.restype = ctypes.c_int
         lib.h3attn_fwd_kv.argtypes = [_P, _P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64_3, _I64_3,
                                       _I64_3, _I64_3, ctypes.c_float, _P, _P]
+        lib.h3attn_qkv_fused.restype = ctypes.c_int
+        lib.h3attn_qkv_fused.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _I64, _I64_3, _I64_3,
+                                         _P, _P, ctypes.c_double, _P, _P, _I32, _I32, _I32, ctypes.c_double, _P]
         lib.h3attn_merge.restype = ctypes.c_int
         lib.h3attn_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I64_3, _I64_3,
                                      _I64_3, _P]
@@ -303,3 +306,47 @@ def merge(o_a, lse_a, o_b, lse_b, o=None, lse=None, stream=None):
     if squeeze:
         return o.squeeze(0), lse.squeeze(0)
     return o, lse
+
+
+def qkv_fused(x, w, n_heads: int, bias=None, q_out=None, k_out=None, v_out=None, gamma_q=None, gamma_k=None,
+              eps: float = 1e-6, pos=None, kind=None, sections: Sequence[int] = (32, 48, 48),
+              theta: float = 10000.0, stream=None):
+    """Q/K/V projection x w^T (+ bias) with RMSNorm + RoPE of Q and K in its epilogue.
+
+    x: bf16 CUDA [n_tokens, dim_in] (last dim contiguous); w: bf16 CUDA [3*H*d, dim_in]
+    contiguous; bias: [3*H*d] or None.  Returns (q, k, v), each [n_tokens, H, d]
+    (new contiguous tensors unless the *_out views are given)."""
+    torch = _torch()
+    _require_bf16_cuda("x", x)
+    _require_bf16_cuda("w", w)
+    if x.dim() != 2 or w.dim() != 2 or w.shape[1] != x.shape[1] or not w.is_contiguous():
+        raise ValueError("x must be [n_tokens, dim_in] and w a contiguous [3*H*d, dim_in]")
+    n, dim_in = x.shape
+    H = int(n_heads)
+    if w.shape[0] % (3 * H):
+        raise ValueError("w must have 3 * n_heads * head_dim rows")
+    d = w.shape[0] // (3 * H)
+    outs = []
+    for name, t in (("q_out", q_out), ("k_out", k_out), ("v_out", v_out)):
+        if t is None:
+            t = torch.empty((n, H, d), dtype=x.dtype, device=x.device)
+        _require_bf16_cuda(name, t)
+        if t.shape != (n, H, d):
+            raise ValueError("%s must be [n_tokens, H, d]" % name)
+        outs.append(t)
+    for name, t in (("bias", bias), ("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        if t is not None:
+            _require_bf16_cuda(name, t)
+    if pos is not None:
+        if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous():
+            raise TypeError("pos must be a contiguous CUDA int32 tensor [n_tokens, 3]")
+        if kind is None or kind.dtype != torch.uint8 or not kind.is_cuda or not kind.is_contiguous():
+            raise TypeError("kind must be a contiguous CUDA uint8 tensor [n_tokens]")
+    st, sh, sw = sections
+    tok = _I64_3(*(max(t.stride(0), 8) if n <= 1 else t.stride(0) for t in outs))
+    hst = _I64_3(*(t.stride(1) for t in outs))
+    _check("h3attn_qkv_fused", library().h3attn_qkv_fused(
+        _ptr(x), _ptr(w), _ptr(bias), _ptr(outs[0]), _ptr(outs[1]), _ptr(outs[2]), n, dim_in, H, d,
+        max(x.stride(0), dim_in) if n <= 1 else x.stride(0), tok, hst, _ptr(gamma_q), _ptr(gamma_k), float(eps),
+        _ptr(pos), _ptr(kind), st, sh, sw, float(theta), _stream_handle(stream)))
+    return tuple(outs)

@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "merge.cuh"
 #include "prologue.cuh"
+#include "qkv.cuh"
 
 namespace {
 
@@ -130,6 +131,54 @@ h3attn_status check_strides(const int64_t* s, int n, const char* name) {
   return H3ATTN_OK;
 }
 
+// Rotary tables shared by the prologue and the fused projection: pair p of the 3D
+// layout belongs to section ax at pair index i inside it, with frequency
+// theta^(-2i/width); 1D tokens use theta^(-2p/d) over all pairs.
+h3attn_status rope_tables(h3::RopeTables* rope, const uint8_t* kind, int head_dim, int sec_t, int sec_h,
+                          int sec_w, double theta) {
+  if (!kind) return fail(H3ATTN_ERR_INVALID_ARG, "kind is required with pos");
+  if (sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t | sec_h | sec_w) & 1 || sec_t + sec_h + sec_w != head_dim)
+    return fail(H3ATTN_ERR_INVALID_ARG, "sections %d/%d/%d must be even and sum to head_dim %d", sec_t, sec_h,
+                sec_w, head_dim);
+  if (!(theta > 0.0) || !std::isfinite(theta)) return fail(H3ATTN_ERR_INVALID_ARG, "theta must be > 0");
+  const int widths[3] = {sec_t, sec_h, sec_w};
+  int pair = 0;
+  for (int ax = 0; ax < 3; ++ax) {
+    for (int i = 0; i < widths[ax] / 2; ++i, ++pair) {
+      rope->axis_3d[pair] = static_cast<uint8_t>(ax);
+      rope->inv_freq_3d[pair] = std::exp(-(2.0 * i / widths[ax]) * std::log(theta));
+    }
+  }
+  for (int i = 0; i < head_dim / 2; ++i) rope->inv_freq_1d[i] = std::exp(-(2.0 * i / head_dim) * std::log(theta));
+  return H3ATTN_OK;
+}
+
+// A row-major bf16 matrix [rows][cols] (row stride in elements) as a tensor map
+// with 64-column x box_rows boxes and 128-byte swizzle (the K-major operand tiles
+// of the projection GEMM).  Rows past the end read as zeros.
+h3attn_status make_map_rows(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t row_stride,
+                            int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(H3ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), 1, 1};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(row_stride) * 2, static_cast<cuuint64_t>(row_stride) * 2 * rows,
+                           static_cast<cuuint64_t>(row_stride) * 2 * rows};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(H3ATTN_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return H3ATTN_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
 float resolve_scale(float scale, int d) {
   const float s = scale > 0.0f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   return static_cast<float>(static_cast<double>(s) * 1.4426950408889634074);
@@ -195,24 +244,7 @@ h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, v
 
   h3::PrologueParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  if (pos) {
-    if (!kind) return fail(H3ATTN_ERR_INVALID_ARG, "kind is required with pos");
-    if (sec_t < 0 || sec_h < 0 || sec_w < 0 || (sec_t | sec_h | sec_w) & 1 || sec_t + sec_h + sec_w != head_dim)
-      return fail(H3ATTN_ERR_INVALID_ARG, "sections %d/%d/%d must be even and sum to head_dim %d", sec_t,
-                  sec_h, sec_w, head_dim);
-    if (!(theta > 0.0) || !std::isfinite(theta)) return fail(H3ATTN_ERR_INVALID_ARG, "theta must be > 0");
-    // rotary tables: pair p of the 3D layout belongs to section ax at pair index i inside it
-    const int widths[3] = {sec_t, sec_h, sec_w};
-    int pair = 0;
-    for (int ax = 0; ax < 3; ++ax) {
-      for (int i = 0; i < widths[ax] / 2; ++i, ++pair) {
-        prm.rope.axis_3d[pair] = static_cast<uint8_t>(ax);
-        prm.rope.inv_freq_3d[pair] = std::exp(-(2.0 * i / widths[ax]) * std::log(theta));
-      }
-    }
-    for (int i = 0; i < head_dim / 2; ++i)
-      prm.rope.inv_freq_1d[i] = std::exp(-(2.0 * i / head_dim) * std::log(theta));
-  }
+  if (pos && (st = rope_tables(&prm.rope, kind, head_dim, sec_t, sec_h, sec_w, theta)) != H3ATTN_OK) return st;
   if (n_tokens == 0) return H3ATTN_OK;
   prm.q_in = static_cast<const uint16_t*>(q_in);
   prm.k_in = static_cast<const uint16_t*>(k_in);
@@ -399,6 +431,78 @@ h3attn_status h3attn_fwd_varlen(const void* q, const void* k, const void* v, voi
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return head_dim == 128 ? launch_attention<128, true>(mq, mk, mv, prm, grid, s)
                          : launch_attention<64, true>(mq, mk, mv, prm, grid, s);
+}
+
+h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, void* q_out, void* k_out,
+                               void* v_out, int64_t n_tokens, int32_t dim_in, int32_t n_heads, int32_t head_dim,
+                               int64_t x_tok_stride, const int64_t out_tok_strides[3],
+                               const int64_t out_head_strides[3], const void* gamma_q, const void* gamma_k,
+                               double eps, const int32_t* pos, const uint8_t* kind, int32_t sec_t, int32_t sec_h,
+                               int32_t sec_w, double theta, void* stream) {
+  if (!x || !w || !q_out || !k_out || !v_out) return fail(H3ATTN_ERR_INVALID_ARG, "null tensor pointer");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(H3ATTN_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (n_tokens < 0 || n_tokens > (int64_t(1) << 31) - h3::kGemmBM)
+    return fail(H3ATTN_ERR_INVALID_ARG, "n_tokens must be in [0, 2^31 - 128]");
+  if (n_heads <= 0 || (static_cast<int64_t>(n_heads) * head_dim) % h3::kGemmBN != 0 ||
+      static_cast<int64_t>(n_heads) * head_dim > (1 << 20))
+    return fail(H3ATTN_ERR_UNSUPPORTED, "n_heads * head_dim must be a positive multiple of %d", h3::kGemmBN);
+  if (dim_in <= 0 || dim_in % h3::kGemmBK != 0 || dim_in > (1 << 20))
+    return fail(H3ATTN_ERR_UNSUPPORTED, "dim_in must be a positive multiple of %d", h3::kGemmBK);
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q_out) || !aligned16(k_out) || !aligned16(v_out) ||
+      (bias && !aligned16(bias)) || (gamma_q && !aligned16(gamma_q)) || (gamma_k && !aligned16(gamma_k)))
+    return fail(H3ATTN_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+  if (x_tok_stride < dim_in) return fail(H3ATTN_ERR_INVALID_ARG, "x_tok_stride must be >= dim_in");
+  h3attn_status st;
+  if ((st = check_strides(&x_tok_stride, 1, "x")) != H3ATTN_OK) return st;
+  if ((st = check_strides(out_tok_strides, 3, "output token")) != H3ATTN_OK) return st;
+  if ((st = check_strides(out_head_strides, 3, "output head")) != H3ATTN_OK) return st;
+  if (!(eps >= 0.0) || !std::isfinite(eps)) return fail(H3ATTN_ERR_INVALID_ARG, "eps must be finite and >= 0");
+
+  h3::QkvParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (pos && (st = rope_tables(&prm.rope, kind, head_dim, sec_t, sec_h, sec_w, theta)) != H3ATTN_OK) return st;
+  if (n_tokens == 0) return H3ATTN_OK;
+  const int64_t features = 3 * static_cast<int64_t>(n_heads) * head_dim;
+  CUtensorMap mx, mw;
+  if ((st = make_map_rows(&mx, x, dim_in, n_tokens, x_tok_stride, h3::kGemmBM)) != H3ATTN_OK) return st;
+  if ((st = make_map_rows(&mw, w, dim_in, features, dim_in, h3::kGemmBN)) != H3ATTN_OK) return st;
+  void* outs[3] = {q_out, k_out, v_out};
+  for (int i = 0; i < 3; ++i) {
+    prm.out[i] = static_cast<uint16_t*>(outs[i]);
+    prm.out_tok[i] = out_tok_strides[i];
+    prm.out_head[i] = out_head_strides[i];
+  }
+  prm.bias = static_cast<const uint16_t*>(bias);
+  prm.gamma[0] = static_cast<const uint16_t*>(gamma_q);
+  prm.gamma[1] = static_cast<const uint16_t*>(gamma_k);
+  prm.pos = pos;
+  prm.kind = kind;
+  prm.n_tokens = n_tokens;
+  prm.dim_in = dim_in;
+  prm.n_heads = n_heads;
+  prm.eps = static_cast<float>(eps);
+  prm.m_tiles = static_cast<int32_t>((n_tokens + h3::kGemmBM - 1) / h3::kGemmBM);
+  prm.n_tiles = static_cast<int32_t>(features / h3::kGemmBN);
+  if (static_cast<int64_t>(prm.m_tiles) * prm.n_tiles > 0x7FFFFFFF)
+    return fail(H3ATTN_ERR_UNSUPPORTED, "too many tiles");
+  prm.ctl.launch_id = next_launch_id();
+  const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
+  const unsigned grid = static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count());
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (head_dim == 128) {
+    e = ensure_smem_attr(h3::qkv_fused_kernel<128>, h3::QkvTraits::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv)");
+    h3::qkv_fused_kernel<128><<<grid, h3::kGemmThreads, h3::QkvTraits::kSmemBytes, s>>>(mx, mw, prm);
+  } else {
+    e = ensure_smem_attr(h3::qkv_fused_kernel<64>, h3::QkvTraits::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv)");
+    h3::qkv_fused_kernel<64><<<grid, h3::kGemmThreads, h3::QkvTraits::kSmemBytes, s>>>(mx, mw, prm);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "qkv launch");
+  return H3ATTN_OK;
 }
 
 }  // extern "C"
