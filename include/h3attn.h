@@ -234,8 +234,10 @@ h3attn_status h3attn_merge(const void* o_a, const float* lse_a, const void* o_b,
  * Requirements: head_dim 64 or 128; n_heads*head_dim a multiple of 256;
  *   dim_in a positive multiple of 64; n_tokens >= 0 (0 is a no-op).
  * Arithmetic: bf16 tensor-core products with fp32 accumulation; bias, sum of
- *   squares, 1/rms (rsqrtf) and the gamma scale in fp32; RoPE with fp64 angles
- *   whose cosine and sine are carried as float pairs and error-free products.
+ *   squares, 1/rms (rsqrtf) and the gamma scale in fp32; RoPE angles formed and
+ *   reduced to [-pi, pi] in fp32 with error-free products (frequencies and 2 pi
+ *   carried as float pairs), cos/sin and the rotation in fp32: about 1e-6
+ *   absolute on cos/sin, far below the accumulation error of the projection.
  */
 h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, void* q_out, void* k_out,
                                void* v_out, int64_t n_tokens, int32_t dim_in, int32_t n_heads,

@@ -8,8 +8,9 @@ the fp32 accumulator across dim_in / 16 accumulation steps with room to spare).
 The norm divides by the row's rms and multiplies by gamma, which carries that
 error over (to first order) as
   |dy_i| <= gamma_i / rms * KAPPA * A_i + |y_i| * KAPPA * sum_j |x_j| A_j / sum_j x_j^2,
-plus a few fp32 roundings of y_i (NORM_REL); the rotation mixes each pair, so a
-rotated element may carry both errors of its pair.  Every output must lie within
+plus a few fp32 roundings of y_i (NORM_REL) and the fp32 rotation (cos/sin within
+2^-21, ROPE_ABS); the rotation mixes each pair, so a rotated element may carry
+both errors of its pair.  Every output must lie within
 half a bf16 ulp of the exact (oracle) value plus that bound."""
 import numpy as np
 import pytest
@@ -22,6 +23,7 @@ pytestmark = pytest.mark.gpu
 
 KAPPA = 2.0 ** -20
 NORM_REL = 2.0 ** -20
+ROPE_ABS = 2.0 ** -19      # fp32 cos/sin (< 2^-21 absolute) and the fp32 rotation, per pair element
 
 
 @pytest.fixture(scope="module")
@@ -67,7 +69,7 @@ def _bounds(x, w, b, rows, H, d, gam, part, y64, pre64):
     rms = np.sqrt(ss / d + 1e-6)
     lin = g / rms * KAPPA * A
     glob = np.abs(pre * g / rms) * KAPPA * np.sum(np.abs(pre) * A, axis=-1, keepdims=True) / ss
-    e = lin + glob + NORM_REL * np.abs(pre * g / rms)
+    e = lin + glob + NORM_REL * np.abs(pre * g / rms) + ROPE_ABS * np.abs(pre * g / rms)
     # RoPE mixes the pair
     pair = e.reshape(len(rows), H, d // 2, 2).sum(-1, keepdims=True)
     return np.broadcast_to(pair, (len(rows), H, d // 2, 2)).reshape(len(rows), H, d)

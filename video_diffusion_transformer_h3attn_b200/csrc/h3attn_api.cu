@@ -461,7 +461,18 @@ h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, v
 
   h3::QkvParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  if (pos && (st = rope_tables(&prm.rope, kind, head_dim, sec_t, sec_h, sec_w, theta)) != H3ATTN_OK) return st;
+  if (pos) {
+    h3::RopeTables rope;
+    std::memset(&rope, 0, sizeof(rope));
+    if ((st = rope_tables(&rope, kind, head_dim, sec_t, sec_h, sec_w, theta)) != H3ATTN_OK) return st;
+    for (int i = 0; i < h3::kRopeMaxPairs; ++i) {  // float pairs: hi + lo = the double to ~2^-48
+      prm.rope.hi3[i] = static_cast<float>(rope.inv_freq_3d[i]);
+      prm.rope.lo3[i] = static_cast<float>(rope.inv_freq_3d[i] - static_cast<double>(prm.rope.hi3[i]));
+      prm.rope.hi1[i] = static_cast<float>(rope.inv_freq_1d[i]);
+      prm.rope.lo1[i] = static_cast<float>(rope.inv_freq_1d[i] - static_cast<double>(prm.rope.hi1[i]));
+      prm.rope.axis3[i] = rope.axis_3d[i];
+    }
+  }
   if (n_tokens == 0) return H3ATTN_OK;
   const int64_t features = 3 * static_cast<int64_t>(n_heads) * head_dim;
   CUtensorMap mx, mw;

@@ -22,10 +22,13 @@
 //     (2 x 256 columns) so the epilogue of one tile overlaps the next tile's
 //     main loop;
 //   * warps 2-9 -- epilogue: a warp owns 32 token rows (its tensor-memory lane
-//     quarter) and 128 of the tile's 256 features; each thread one token row.
-//     Q/K heads: sum of squares and RMS in fp32, x * (1/rms) * gamma, then RoPE
-//     with cos/sin of fp64 angles carried as float pairs and error-free
-//     products (as the standalone prologue); V: bias and rounding only.
+//     quarter) and 128 of the tile's 256 features; each thread one token row,
+//     32 accumulator columns at a time (a first pass over a Q/K head forms the
+//     sum of squares).  Q/K heads: RMS in fp32, x * (1/rms) * gamma, then RoPE
+//     with the angle formed and reduced to [-pi, pi] in fp64 and cos/sin from
+//     the fp32 intrinsic (the projection's fp32 accumulation error dominates
+//     here, unlike in the standalone prologue whose input is exact); V: bias and
+//     rounding only.
 // Tiles are numbered feature-tile fastest, so the CTAs running at once share a
 // few X row blocks and W stays resident in L2 (3*H*d x dim_in bf16 = 57 MB at
 // H*d = dim_in = 3072).  Every barrier wait is bounded (common.cuh).
@@ -48,6 +51,15 @@ constexpr int kGemmThreads = 320;
 constexpr int kGemmEpiWarp0 = 2;  // warps 2..9: epilogue
 constexpr int kGemmEpiWarps = 8;
 
+// Rotary frequencies as float pairs (hi + lo = the fp64 value to ~2^-48): the
+// epilogue forms p * f and reduces it modulo 2 pi in fp32 arithmetic with
+// error-free products, without fp64 (which is slow on this part).
+struct RopeTablesF {
+  float hi3[kRopeMaxPairs], lo3[kRopeMaxPairs];  // 3D layout, pair p inside its section
+  float hi1[kRopeMaxPairs], lo1[kRopeMaxPairs];  // 1D layout
+  uint8_t axis3[kRopeMaxPairs];                  // 0 = t, 1 = h, 2 = w
+};
+
 struct QkvParams {
   uint16_t* out[3];           // Q', K', V (bf16)
   int64_t out_tok[3];         // element strides
@@ -56,7 +68,7 @@ struct QkvParams {
   const uint16_t* gamma[2];   // [d] or null (Q, K)
   const int32_t* pos;         // [n_tokens][3] or null
   const uint8_t* kind;        // [n_tokens]
-  RopeTables rope;
+  RopeTablesF rope;
   int64_t n_tokens;
   int32_t dim_in;
   int32_t n_heads;
@@ -218,60 +230,110 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
       for (int h0 = 0; h0 < 128; h0 += D) {      // the heads among this warp's 128 features
         const int head = (f0 + h0 - part * hd) / D;
-        float x[D];
+        const uint4* const bias4 = p.bias ? reinterpret_cast<const uint4*>(p.bias + f0 + h0) : nullptr;
+        const bool norm = part < 2 && p.gamma[part] != nullptr;
+        // bias of 32 columns starting at c, added to v; 16-byte loads at the same
+        // addresses in every thread (served once per warp)
+        auto add_bias = [&](int c, float* v) {
+          if (bias4) {
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tacc + h0 + c, r);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 bv = __ldg(bias4 + c / 8 + q);
+              const uint32_t w4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                v[8 * q + 2 * i] += __uint_as_float(w4[i] << 16);
+                v[8 * q + 2 * i + 1] += __uint_as_float(w4[i] & 0xFFFF0000u);
+              }
+            }
+          }
+        };
+        // pass 1 (Q, K): the row's sum of squares -- all of the head's columns in
+        // flight at once, one wait; they are read again below
+        float rinv = 1.0f;
+        if (norm) {
+          uint32_t ra[D / 32][32];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(tacc + h0 + 32 * c, ra[c]);
           ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) x[c + i] = __uint_as_float(r[i]);
-        }
-        if (p.bias) {
-          const uint16_t* b = p.bias + f0 + h0;
-#pragma unroll
-          for (int i = 0; i < D; ++i) x[i] += __uint_as_float(static_cast<uint32_t>(b[i]) << 16);
-        }
-        if (part < 2 && p.gamma[part]) {
           float ss = 0.0f;
 #pragma unroll
-          for (int i = 0; i < D; ++i) ss = fmaf(x[i], x[i], ss);
-          const float r = rsqrtf(ss / static_cast<float>(D) + p.eps);
-          const uint16_t* g = p.gamma[part];
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
 #pragma unroll
-          for (int i = 0; i < D; ++i) x[i] = (x[i] * r) * __uint_as_float(static_cast<uint32_t>(g[i]) << 16);
-        }
-        if (rope) {
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ra[c][i]);
+            add_bias(32 * c, v);
 #pragma unroll
-          for (int pr = 0; pr < D / 2; ++pr) {
-            double angle;
-            if (kd == 1) {
-              const int ax = p.rope.axis_3d[pr];
-              angle = static_cast<double>(ax == 0 ? pt0 : ax == 1 ? pt1 : pt2) * p.rope.inv_freq_3d[pr];
-            } else {
-              angle = static_cast<double>(pt0) * p.rope.inv_freq_1d[pr];
-            }
-            double sd, cd;
-            sincos(angle, &sd, &cd);
-            const float ch = static_cast<float>(cd), cl = static_cast<float>(cd - static_cast<double>(ch));
-            const float sh = static_cast<float>(sd), sl = static_cast<float>(sd - static_cast<double>(sh));
-            const float a0 = x[2 * pr], a1 = x[2 * pr + 1];
-            const float p0 = a0 * ch, e0 = fmaf(a0, ch, -p0);
-            const float q0 = a1 * sh, g0 = fmaf(a1, sh, -q0);
-            const float p1 = a0 * sh, e1 = fmaf(a0, sh, -p1);
-            const float q1 = a1 * ch, g1 = fmaf(a1, ch, -q1);
-            x[2 * pr] = (p0 - q0) + (fmaf(a0, cl, e0) - fmaf(a1, sl, g0));
-            x[2 * pr + 1] = (p1 + q1) + (fmaf(a0, sl, e1) + fmaf(a1, cl, g1));
+            for (int i = 0; i < 32; ++i) ss = fmaf(v[i], v[i], ss);
           }
+          rinv = rsqrtf(ss / static_cast<float>(D) + p.eps);
         }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out[part] + n * p.out_tok[part] +
-                                                static_cast<int64_t>(head) * p.out_head[part]);
+        // pass 2: scale, rotate, round, store -- 64 columns per wait, 32 at a time
+        uint4* const dst = reinterpret_cast<uint4*>(p.out[part] + (valid ? n : 0) * p.out_tok[part] +
+                                                    static_cast<int64_t>(head) * p.out_head[part]);
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            dst[c] = make_uint4(ptx::pack_bf16x2(x[8 * c], x[8 * c + 1]), ptx::pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
-                                ptx::pack_bf16x2(x[8 * c + 4], x[8 * c + 5]),
-                                ptx::pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
+        for (int c2 = 0; c2 < D; c2 += 64) {
+          uint32_t rb[2][32];
+          ptx::tmem_ld32(tacc + h0 + c2, rb[0]);
+          ptx::tmem_ld32(tacc + h0 + c2 + 32, rb[1]);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int c = c2 + 32 * hh;
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rb[hh][i]);
+            add_bias(c, v);
+            if (norm) {
+              const uint4* g = reinterpret_cast<const uint4*>(p.gamma[part]) + c / 8;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 gv = __ldg(g + q);
+                const uint32_t w4[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  v[8 * q + 2 * i] = (v[8 * q + 2 * i] * rinv) * __uint_as_float(w4[i] << 16);
+                  v[8 * q + 2 * i + 1] = (v[8 * q + 2 * i + 1] * rinv) * __uint_as_float(w4[i] & 0xFFFF0000u);
+                }
+              }
+            }
+            if (rope) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int pr = c / 2 + i;  // rotation pair of columns (2 pr, 2 pr + 1)
+                float pf, fh, fl;          // position (exact) and frequency hi + lo
+                if (kd == 1) {
+                  const int ax = p.rope.axis3[pr];
+                  pf = static_cast<float>(ax == 0 ? pt0 : ax == 1 ? pt1 : pt2);
+                  fh = p.rope.hi3[pr];
+                  fl = p.rope.lo3[pr];
+                } else {
+                  pf = static_cast<float>(pt0);
+                  fh = p.rope.hi1[pr];
+                  fl = p.rope.lo1[pr];
+                }
+                // angle = pf * (fh + fl) as prod + tail (prod + e exact), reduced modulo
+                // 2 pi (2 pi as hi + lo): |error| ~ 2^-24 pi + |angle| 2^-46 before cos/sin
+                const float prod = pf * fh;
+                const float tail = fmaf(pf, fh, -prod) + pf * fl;
+                const float turns = rintf(prod * 0.159154943091895336f);
+                float red = fmaf(-turns, 6.28318548202514648f, prod);   // 2 pi rounded to float
+                red = fmaf(-turns, -1.74845553e-7f, red) + tail;           // 2 pi = that + this
+                float sn, cs;
+                __sincosf(red, &sn, &cs);
+                const float a0 = v[2 * i], a1 = v[2 * i + 1];
+                v[2 * i] = fmaf(a0, cs, -a1 * sn);
+                v[2 * i + 1] = fmaf(a0, sn, a1 * cs);
+              }
+            }
+            if (valid) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                dst[c / 8 + q] = make_uint4(ptx::pack_bf16x2(v[8 * q], v[8 * q + 1]), ptx::pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                            ptx::pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                            ptx::pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+              }
+            }
           }
         }
       }
