@@ -489,25 +489,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       };
       uint32_t pk[16];
       // First half (keys 0..63) with the running max m as it stands, while this
-      // tile's row maxima are formed beside it on another pipe.  Only where a max
+      // tile's row maxima are formed beside it on another pipe (the max chains are
+      // interleaved with the exponentials in the issue order).  Only where a max
       // grows by more than the threshold (always at j = 0, rarely later) are m and
       // that half redone, so the max is off the critical path of the step.
+      float a0 = fmaxf(s0[0], s0[1]), b0 = fmaxf(s0[2], s0[3]);
+      float a1 = fmaxf(s1[0], s1[1]), b1 = fmaxf(s1[2], s1[3]);
       {
         const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < 8; ++k) {
           p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, k, pk[2 * k], pk[2 * k + 1]);
+          if (k < 7) {
+            const int e = 4 * (k + 1);
+            a0 = ptx::max3(a0, s0[e], s0[e + 1]);
+            b0 = ptx::max3(b0, s0[e + 2], s0[e + 3]);
+            a1 = ptx::max3(a1, s1[e], s1[e + 1]);
+            b1 = ptx::max3(b1, s1[e + 2], s1[e + 3]);
+          }
+        }
       }
-      // row maxima: this thread's 32 keys, then the quad
-      float a0 = fmaxf(s0[0], s0[1]), b0 = fmaxf(s0[2], s0[3]);
-      float a1 = fmaxf(s1[0], s1[1]), b1 = fmaxf(s1[2], s1[3]);
-#pragma unroll
-      for (int e = 4; e < 32; e += 4) {
-        a0 = ptx::max3(a0, s0[e], s0[e + 1]);
-        b0 = ptx::max3(b0, s0[e + 2], s0[e + 3]);
-        a1 = ptx::max3(a1, s1[e], s1[e + 1]);
-        b1 = ptx::max3(b1, s1[e + 2], s1[e + 3]);
-      }
+      // row maxima: this thread's 32 keys (above), then the quad's four threads
       float mx0 = fmaxf(a0, b0), mx1 = fmaxf(a1, b1);
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
