@@ -24,7 +24,8 @@
 //   * warps 2-9 -- epilogue: a warp owns 32 token rows (its tensor-memory lane
 //     quarter) and 128 of the tile's 256 features; each thread one token row,
 //     32 accumulator columns at a time (a first pass over a Q/K head forms the
-//     sum of squares).  Q/K heads: RMS in fp32, x * (1/rms) * gamma, then RoPE
+//     sum of squares); results go through a per-warp 2 KB shared-memory block
+//     so that four lanes write each row's 64 bytes together.  Q/K heads: RMS in fp32, x * (1/rms) * gamma, then RoPE
 //     with the angle formed and reduced to [-pi, pi] in fp64 and cos/sin from
 //     the fp32 intrinsic (the projection's fp32 accumulation error dominates
 //     here, unlike in the standalone prologue whose input is exact); V: bias and
@@ -83,7 +84,11 @@ struct QkvTraits {
   static constexpr int kStageBytes = kABytes + kBBytes;
   // barriers: full[S], empty[S], acc_full[2], acc_empty[2]
   static constexpr int kBarriers = 2 * kGemmStages + 4;
-  static constexpr int kSmemBytes = 1024 + kGemmStages * kStageBytes + 8 * kBarriers + 16;
+  // per epilogue warp: a 32-row x 32-column bf16 staging block (2 KB) that turns
+  // its thread-per-row results into row-contiguous global stores
+  static constexpr int kStageOutBytes = 32 * 32 * 2;
+  static constexpr int kSmemBytes =
+      1024 + kGemmStages * kStageBytes + 8 * kBarriers + 16 + kGemmEpiWarps * kStageOutBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -104,6 +109,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto bar_acc_full = [&](int b) { return bars + 8u * (2 * kS + b); };
   auto bar_acc_empty = [&](int b) { return bars + 8u * (2 * kS + 2 + b); };
   volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + 8 * T::kBarriers);
+  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + 8 * T::kBarriers + 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -203,6 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quarter = warp & 3;          // tensor-memory lane quarter of this warp
     const int half = ew >> 2;              // which 128 of the tile's 256 features
     const int row = quarter * 32 + lane;   // token row inside the tile
+    uint8_t* const wstage = stage_out + ew * T::kStageOutBytes;
     const int hd = p.n_heads * D;
     bool ok = true;
     int k = 0;
@@ -269,8 +276,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           rinv = rsqrtf(ss / static_cast<float>(D) + p.eps);
         }
         // pass 2: scale, rotate, round, store -- 64 columns per wait, 32 at a time
-        uint4* const dst = reinterpret_cast<uint4*>(p.out[part] + (valid ? n : 0) * p.out_tok[part] +
-                                                    static_cast<int64_t>(head) * p.out_head[part]);
 #pragma unroll
         for (int c2 = 0; c2 < D; c2 += 64) {
           uint32_t rb[2][32];
@@ -326,14 +331,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 v[2 * i + 1] = fmaf(a0, sn, a1 * cs);
               }
             }
-            if (valid) {
+            // stage this thread's 32 columns (four 16-byte pieces of its row) in the
+            // warp's block, pieces swizzled by row so that the writes and the
+            // row-wise reads below are free of bank conflicts
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                dst[c / 8 + q] = make_uint4(ptx::pack_bf16x2(v[8 * q], v[8 * q + 1]), ptx::pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                            ptx::pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                            ptx::pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            for (int q = 0; q < 4; ++q) {
+              const int sw = q ^ ((lane >> 1) & 3);
+              *reinterpret_cast<uint4*>(wstage + lane * 64 + sw * 16) =
+                  make_uint4(ptx::pack_bf16x2(v[8 * q], v[8 * q + 1]), ptx::pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                             ptx::pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), ptx::pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            }
+            __syncwarp();
+            // row-contiguous stores: lanes 4r..4r+3 write the 64 bytes of one row
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              const int srow = rr * 8 + (lane >> 2), piece = lane & 3;
+              const int64_t tok = static_cast<int64_t>(m) * kGemmBM + quarter * 32 + srow;
+              const uint4 val =
+                  *reinterpret_cast<const uint4*>(wstage + srow * 64 + (piece ^ ((srow >> 1) & 3)) * 16);
+              if (tok < p.n_tokens) {
+                uint16_t* const drow = p.out[part] + tok * p.out_tok[part] +
+                                       static_cast<int64_t>(head) * p.out_head[part] + c;
+                *reinterpret_cast<uint4*>(drow + piece * 8) = val;
               }
             }
+            __syncwarp();  // the block is reused by the next 32 columns
           }
         }
       }
