@@ -208,12 +208,14 @@ ATTENTION_SOURCES = ("attention.cuh", "sm100_ptx.cuh", "common.cuh")
 
 
 def source_hash():
-    """Hash of the attention kernel's sources (a stored ncu figure is only used
-    while these are unchanged)."""
+    """Hash of the attention kernel's sources with comments and blank space
+    removed (a stored ncu figure is only used while the code is unchanged)."""
+    import re
     h = hashlib.sha256()
     for f in ATTENTION_SOURCES:
-        with open(os.path.join(ROOT, "video_diffusion_transformer_h3attn_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "video_diffusion_transformer_h3attn_b200", "csrc", f)) as fh:
+            text = re.sub(r"//[^\n]*", "", fh.read())
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -5,7 +5,10 @@
  *
  * The path: per-head Q/K RMSNorm + rotary position embedding (one prologue
  * kernel), then non-causal softmax(Q K^T * scale) V over a packed token
- * sequence (one attention kernel, dense or ragged).
+ * sequence (one attention kernel, dense or ragged).  Around it: attention
+ * against a separate key block and the log-sum-exp merge of such partial
+ * results (key-split schedules), and the Q/K/V projection with the prologue
+ * fused into its epilogue.
  *
  * Sources of the operations (web pages about the H3 runtimes):
  *   - "H3 Runtime Current State", Owned Performance Kernels: a fused Q/K

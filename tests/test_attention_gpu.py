@@ -136,3 +136,36 @@ def test_special_cases(h3, orc):
     o, _ = _gpu_dense(h3, w.q, w.k, vc)
     check_attention(bf16_bits_to_f64(o), bf16_bits_to_f64(vc), "constant V")
     assert np.mean(o == vc) > 0.99, "constant V rows should come back (almost always) exactly"
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_many_sequences(h3, orc, d):
+    """More sequences than the in-kernel longest-first ranking takes (256): the
+    launch falls back to the given order, with empty and one-token sequences."""
+    rng = np.random.default_rng(77 + d)
+    lens = rng.integers(0, 200, size=300)
+    lens[::37] = 0
+    lens[5] = 1
+    w = inputs.random_case(list(int(x) for x in lens), 2, d, seed=960 + d)
+    o, lse = _gpu_varlen(h3, w.q, w.k, w.v, w.cu_seqlens)
+    ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "300 sequences d=%d" % d, lse.T, rl)
+
+
+def test_ragged_schedule_does_not_change_results(h3):
+    """The same sequences give the same bits whether the kernel ranks them
+    longest first (<= 256 sequences) or takes them in the given order (more
+    sequences: 50 empty ones appended), and in a dense launch of one of them."""
+    import torch
+    rng = np.random.default_rng(5)
+    lens = [int(x) for x in rng.integers(1, 400, size=200)]
+    w = inputs.random_case(lens, 2, 128, seed=970)
+    o_sorted, l_sorted = _gpu_varlen(h3, w.q, w.k, w.v, w.cu_seqlens)
+    cu_more = np.concatenate([w.cu_seqlens, np.full(50, w.cu_seqlens[-1], dtype=np.int32)])
+    o_given, l_given = _gpu_varlen(h3, w.q, w.k, w.v, cu_more)
+    assert np.array_equal(o_sorted, o_given), "ranked and given orders must give identical outputs"
+    assert np.array_equal(l_sorted, l_given)
+    s = 17
+    a, b = int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1])
+    o_one, _ = _gpu_dense(h3, w.q[a:b], w.k[a:b], w.v[a:b])
+    assert np.array_equal(o_one, o_sorted[a:b]), "a ragged sequence equals its dense launch bit for bit"

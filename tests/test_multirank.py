@@ -27,7 +27,7 @@ def _worker(rank, world, port, out):
 
 def test_reduce_max_over_two_gloo_ranks():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     assert dict(out) == {0: 125.0, 1: 125.0}
 

@@ -95,7 +95,7 @@ def _one_rank(seqlens, H, d, seed):
 @pytest.mark.parametrize("world,seqlens", [(2, [37]), (3, [37]), (2, [20, 1, 30]), (3, [64])])
 def test_ulysses_matches_one_rank_bit_for_bit(world, seqlens):
     H, d, seed = 6, 16, 11
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, _free_port(), seqlens, H, d, seed, out), nprocs=world, join=True)
     ref = _one_rank(seqlens, H, d, seed)
     off = ulysses.shard_offsets(ulysses.shard_sizes(sum(seqlens), world))
