@@ -6,7 +6,9 @@
 // largest share of the profiled block; "Open-H3-Regenerate-2K", forward table:
 // dense attention on one B200).  Ragged batches follow "H3 Runtime Current
 // State" (ragged sequence parallelism): each cu_seqlens segment attends only to
-// itself.
+// itself, and CTAs take the segments longest first.  Dense launches may give
+// the keys their own length (one block of a split key set: O and LSE are then
+// that block's partial result; no keys at all give O = 0, LSE = -inf).
 //
 // One CTA per SM (640 threads = five warpgroups) owns two 128-row query tiles
 // Q0, Q1 of one (sequence, head):
@@ -97,36 +99,6 @@ __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uin
   }
   return true;
 }
-
-// 2^x for a pair of values x <= 8, on the FMA and integer pipes instead of the
-// exponential unit.  x = n + f with n = rint(x) and f in [-1/2, 1/2]; 2^f by a
-// degree-3 polynomial whose coefficients were fitted for this kernel by a Remez
-// exchange on the relative error (max 7.5e-5 over [-1/2, 1/2], far below the 2^-8
-// of the bf16 rounding that follows); 2^n is added to the exponent field.  x is
-// clamped at -125 so the result stays a normal number (2^-125 where the exact
-// value is smaller, e.g. masked keys: negligible next to a row sum >= 1).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
-  constexpr float kC2 = 0.2426111251115799f, kC3 = 0.0551716685295105f;
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));         // n in the low mantissa bits
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));       // n as a float
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);        // x - n
-  float2 q = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
-  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
-
-// Every kEmuEvery-th pair of exponentials goes through exp2_poly2 (0 = none),
-// moving part of the work from the exponential unit (16/clk/SM) to the FMA pipes.
-#ifndef H3ATTN_EMU_EVERY
-#define H3ATTN_EMU_EVERY 0
-#endif
-constexpr int kEmuEvery = H3ATTN_EMU_EVERY;
 
 template <int D, bool kVarlen, bool kLse>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -465,19 +437,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // keys 8k + 2*cq + {0,1} is packed column 4k + cq (16x128b shape).
       float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
       float2 accx0 = make_float2(0.0f, 0.0f), accx1 = make_float2(0.0f, 0.0f);
-      // one pair of keys (pair index k) for both rows: exponentials, packing, sums
-      auto p_pair = [&](float sa0, float sa1, float sb0, float sb1, float2 nm0, float2 nm1, int k,
-                        uint32_t& pa, uint32_t& pb) {
+      // one pair of keys for both rows: exponentials, packing, sums
+      auto p_pair = [&](float sa0, float sa1, float sb0, float sb1, float2 nm0, float2 nm1, uint32_t& pa,
+                        uint32_t& pb) {
         const float2 x0 = __ffma2_rn(make_float2(sa0, sa1), c2, nm0);
         const float2 x1 = __ffma2_rn(make_float2(sb0, sb1), c2, nm1);
-        float2 e0, e1;
-        if (kEmuEvery > 0 && (k % (kEmuEvery > 0 ? kEmuEvery : 1)) == kEmuEvery - 1) {
-          e0 = exp2_poly2(x0);
-          e1 = exp2_poly2(x1);
-        } else {
-          e0 = make_float2(ptx::ex2_approx(x0.x), ptx::ex2_approx(x0.y));
-          e1 = make_float2(ptx::ex2_approx(x1.x), ptx::ex2_approx(x1.y));
-        }
+        const float2 e0 = make_float2(ptx::ex2_approx(x0.x), ptx::ex2_approx(x0.y));
+        const float2 e1 = make_float2(ptx::ex2_approx(x1.x), ptx::ex2_approx(x1.y));
         pa = ptx::pack_bf16x2(e0.x, e0.y);
         pb = ptx::pack_bf16x2(e1.x, e1.y);
         ptx::add_bf16x2_f32(acc0.x, acc0.y, pa);
@@ -499,7 +465,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float2 nm0 = make_float2(-m0, -m0), nm1 = make_float2(-m1, -m1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, k, pk[2 * k], pk[2 * k + 1]);
+          p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, pk[2 * k], pk[2 * k + 1]);
           if (k < 7) {
             const int e = 4 * (k + 1);
             a0 = ptx::max3(a0, s0[e], s0[e + 1]);
@@ -548,7 +514,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               for (int i = 0; i < 2; ++i)
                 if (8 * k + 2 * cq + i >= kv_last_valid) v[i] = v[2 + i] = -INFINITY;
             }
-            p_pair(v[0], v[1], v[2], v[3], nm0, nm1, k, pk[2 * k], pk[2 * k + 1]);
+            p_pair(v[0], v[1], v[2], v[3], nm0, nm1, pk[2 * k], pk[2 * k + 1]);
           }
         }
       }
@@ -559,7 +525,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const int k = 8 + kk;
-          p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, k, pk[2 * kk], pk[2 * kk + 1]);
+          p_pair(s0[2 * k], s0[2 * k + 1], s1[2 * k], s1[2 * k + 1], nm0, nm1, pk[2 * kk], pk[2 * kk + 1]);
         }
       }
       ptx::tmem_st_16x128b_x8(tS + 32, pk);
