@@ -71,6 +71,9 @@ class Oracle:
                                           _I32, _I32, _I32, _D, _P, _I64, _P, _P, _P, _P, _P, _P]
         lib.h3o_merge.restype = ctypes.c_int
         lib.h3o_merge.argtypes = [_P, _P, _I32, _I64, _I32, _P, _P]
+        lib.h3o_attention_block_sparse.restype = ctypes.c_int
+        lib.h3o_attention_block_sparse.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I32, _I32,
+                                                   _P, _P, _D, _P, _I64, _P, _P]
         self.lib = lib
 
     # -- bfloat16 rounding --------------------------------------------------------
@@ -159,6 +162,42 @@ class Oracle:
                                        _ptr(ck), len(cq) - 1, float(scale), _ptr(o), _ptr(lse))
         if rc != 0:
             raise ValueError("oracle attention_kv rejected its arguments (%d)" % rc)
+        return o, lse
+
+    def attention_block_sparse(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, blk_off, blk_idx,
+                               block_q: int = 256, block_k: int = 128, scale: Optional[float] = None,
+                               rows=None) -> Tuple[np.ndarray, np.ndarray]:
+        """Attention of each query to the keys of the key blocks listed for its
+        (batch, head, query block).
+
+        q: bf16 bits [B, n_q, H, d]; k, v: [B, n_kv, H, d]; blk_off: int32 CSR offsets
+        [B*H*ceil(n_q/block_q) + 1] into blk_idx (key-block indices).  rows: optional
+        flat query rows b*n_q + t.  Returns (o [rows, H, d], lse [rows, H]) with
+        rows = all B*n_q rows when not given; no visible key gives o = 0, lse = -inf."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        B, n_q, H, d = q.shape
+        k = np.ascontiguousarray(k, dtype=np.uint16).reshape(B, -1, H, d)
+        v = np.ascontiguousarray(v, dtype=np.uint16).reshape(B, -1, H, d)
+        n_kv = k.shape[1]
+        off = np.ascontiguousarray(blk_off, dtype=np.int32)
+        idx = np.ascontiguousarray(blk_idx, dtype=np.int32)
+        n_qb = -(-n_q // block_q)
+        if off.shape != (B * H * n_qb + 1,):
+            raise ValueError("blk_off must have B*H*ceil(n_q/block_q) + 1 entries")
+        if idx.size < int(off[-1]):
+            raise ValueError("blk_idx is shorter than blk_off[-1]")
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        rws = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+        nrows = B * n_q if rws is None else rws.size
+        o = np.empty((nrows, H, d), dtype=np.float64)
+        lse = np.empty((nrows, H), dtype=np.float64)
+        rc = self.lib.h3o_attention_block_sparse(
+            _ptr(q), _ptr(k), _ptr(v), B, n_q, n_kv, H, d, block_q, block_k, _ptr(off),
+            _ptr(idx) if idx.size else None, float(scale), None if rws is None else _ptr(rws), nrows,
+            _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle attention_block_sparse rejected its arguments (%d)" % rc)
         return o, lse
 
     def merge(self, o_parts, lse_parts) -> Tuple[np.ndarray, np.ndarray]:

@@ -395,3 +395,96 @@ int h3o_qkv_norm_rope(const uint16_t* x, int64_t n_tokens, int32_t dim_in, int64
     }
     return 0;
 }
+
+/*
+ * Block-sparse attention over a dense batch.  The pages name a sparse attention
+ * backend ("Open-H3-Regenerate-2K", refine timing table: "+ Sol-Attn sparse
+ * attention", lossy and quality-gated per "H3 Runtime Current State", Next Work)
+ * but not its selection rule, so only the execution of a given block pattern is
+ * defined here: the n_q queries of a sequence are cut into query blocks of block_q
+ * rows and its n_kv keys into key blocks of block_k keys; for every (batch b,
+ * head h, query block qb) the list
+ *     blk_idx[blk_off[c] .. blk_off[c + 1]),  c = (b * n_heads + h) * QB + qb,
+ *     QB = ceil(n_q / block_q),
+ * names the key blocks its queries see.  A query attends to exactly the keys of
+ * the listed blocks (keys past n_kv in a listed last block do not exist; a block
+ * listed twice counts once), with the arithmetic of h3o_attention on that key
+ * set; no key at all is the empty sum, o = 0 and lse = -inf.
+ *   q: bf16 bits [batch][n_q][n_heads][d];  k, v: [batch][n_kv][n_heads][d].
+ *   rows: int64 [nrows] query rows b * n_q + t (NULL = all batch * n_q rows).
+ *   o: double [nrows][n_heads][d];  lse: double [nrows][n_heads] or NULL.
+ * Returns 0, or -1 on invalid arguments (offsets not starting at 0 or decreasing,
+ * a block index outside [0, ceil(n_kv / block_k))).
+ */
+int h3o_attention_block_sparse(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               int32_t batch, int64_t n_q, int64_t n_kv, int32_t n_heads, int32_t d,
+                               int32_t block_q, int32_t block_k, const int32_t* blk_off,
+                               const int32_t* blk_idx, double scale, const int64_t* rows,
+                               int64_t nrows, double* o, double* lse) {
+    if (!q || !o || !blk_off || batch <= 0 || n_q < 0 || n_kv < 0 || n_heads <= 0 || d <= 0 ||
+        d > 1024 || block_q <= 0 || block_k <= 0)
+        return -1;
+    if (n_kv > 0 && (!k || !v)) return -1;
+    const int64_t n_qb = (n_q + block_q - 1) / block_q;
+    const int64_t n_kb = (n_kv + block_k - 1) / block_k;
+    const int64_t n_lists = (int64_t)batch * n_heads * n_qb;
+    if (blk_off[0] != 0) return -1;
+    for (int64_t c = 0; c < n_lists; ++c) {
+        if (blk_off[c + 1] < blk_off[c]) return -1;
+        for (int64_t e = blk_off[c]; e < blk_off[c + 1]; ++e)
+            if (!blk_idx || blk_idx[e] < 0 || blk_idx[e] >= n_kb) return -1;
+    }
+    if (!rows) nrows = (int64_t)batch * n_q;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t g = rows ? rows[r] : r;
+        if (g < 0 || g >= (int64_t)batch * n_q) return -1;
+    }
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t g = rows ? rows[r] : r;
+        const int64_t b = g / n_q, t = g % n_q;
+        char* seen = (char*)calloc((size_t)(n_kb > 0 ? n_kb : 1), 1);
+        double* s_row = (double*)malloc(sizeof(double) * (size_t)(n_kv > 0 ? n_kv : 1));
+        for (int h = 0; h < n_heads; ++h) {
+            const int64_t list = ((int64_t)b * n_heads + h) * n_qb + t / block_q;
+            memset(seen, 0, (size_t)(n_kb > 0 ? n_kb : 1));
+            for (int64_t e = blk_off[list]; e < blk_off[list + 1]; ++e) seen[blk_idx[e]] = 1;
+            double qv[1024];
+            for (int i = 0; i < d; ++i)
+                qv[i] = h3o_bf16_to_double(q[((b * n_q + t) * n_heads + h) * (int64_t)d + i]);
+            /* scores of the visible keys, and their maximum */
+            double m = -INFINITY;
+            int64_t n_vis = 0;
+            for (int64_t j = 0; j < n_kv; ++j) {
+                if (!seen[j / block_k]) continue;
+                const int64_t kr = ((b * n_kv + j) * n_heads + h) * (int64_t)d;
+                double qk = 0.0;
+                for (int i = 0; i < d; ++i) qk += qv[i] * h3o_bf16_to_double(k[kr + i]);
+                s_row[j] = scale * qk;
+                if (s_row[j] > m) m = s_row[j];
+                ++n_vis;
+            }
+            double* row_o = o + (r * n_heads + h) * (int64_t)d;
+            if (n_vis == 0) {  /* no key: the empty sum */
+                for (int i = 0; i < d; ++i) row_o[i] = 0.0;
+                if (lse) lse[r * n_heads + h] = -INFINITY;
+                continue;
+            }
+            double num[1024];
+            for (int i = 0; i < d; ++i) num[i] = 0.0;
+            double z = 0.0;
+            for (int64_t j = 0; j < n_kv; ++j) {
+                if (!seen[j / block_k]) continue;
+                const int64_t vr = ((b * n_kv + j) * n_heads + h) * (int64_t)d;
+                const double wgt = exp(s_row[j] - m);
+                z += wgt;
+                for (int i = 0; i < d; ++i) num[i] += wgt * h3o_bf16_to_double(v[vr + i]);
+            }
+            for (int i = 0; i < d; ++i) row_o[i] = num[i] / z;
+            if (lse) lse[r * n_heads + h] = m + log(z);
+        }
+        free(seen);
+        free(s_row);
+    }
+    return 0;
+}

@@ -20,6 +20,10 @@ What pins what:
                   the mean of V; one key gives V_0; constant V; permutation
                   invariance; a dominant key; isolation between sequences;
                   sampled rows equal full rows.
+  block-sparse    torch scaled_dot_product_attention in float64 with the
+                  boolean mask the block lists describe (built by plain loops);
+                  all blocks listed equals unmasked attention; rows with no
+                  key give the empty sum.
 """
 from __future__ import annotations
 
@@ -502,6 +506,73 @@ def pin_qkv_projection(orc):
     _close(qs, q[rows], 0, 0, "sampled rows")
 
 
+def _block_mask(B, H, n_q, n_kv, block_q, block_k, off, idx):
+    """Boolean [B, H, n_q, n_kv] visibility from CSR block lists, by direct loops."""
+    n_qb = -(-n_q // block_q)
+    mask = np.zeros((B, H, n_q, n_kv), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            for qb in range(n_qb):
+                c = (b * H + h) * n_qb + qb
+                for e in range(int(off[c]), int(off[c + 1])):
+                    kb = int(idx[e])
+                    mask[b, h, qb * block_q:(qb + 1) * block_q, kb * block_k:(kb + 1) * block_k] = True
+    return mask
+
+
+def pin_attention_block_sparse(orc):
+    """Block-sparse attention against torch scaled_dot_product_attention in
+    float64 with the equivalent boolean mask (lists unsorted, with repeats and
+    empty ones; a partial last key block; n_q != n_kv); all blocks listed equals
+    plain attention; rows that see no key give o = 0, lse = -inf."""
+    rng = np.random.default_rng(23)
+    B, H, n_q, n_kv, d = 2, 2, 37, 29, 16
+    bq, bk = 6, 8  # slips that swap the two sizes stay inside the buffers
+    n_qb, n_kb = -(-n_q // bq), -(-n_kv // bk)
+    q = to_bf16_bits_f32(rng.standard_normal((B, n_q, H, d)))
+    k = to_bf16_bits_f32(rng.standard_normal((B, n_kv, H, d)))
+    v = to_bf16_bits_f32(rng.standard_normal((B, n_kv, H, d)))
+    lists = []
+    for c in range(B * H * n_qb):
+        n = int(rng.integers(0, n_kb + 2)) if c % 5 else 0
+        lists.append(list(rng.integers(0, n_kb, size=n)))
+    off = np.concatenate([[0], np.cumsum([len(x) for x in lists])]).astype(np.int32)
+    idx = np.array([e for x in lists for e in x], dtype=np.int32)
+    scale = 0.29
+    o, lse = orc.attention_block_sparse(q, k, v, off, idx, bq, bk, scale)
+    mask = _block_mask(B, H, n_q, n_kv, bq, bk, off, idx)
+    qt, kt, vt = (torch.from_numpy(bf16_value(a)).permute(0, 2, 1, 3) for a in (q, k, v))
+    s = torch.einsum("bhnd,bhmd->bhnm", qt, kt) * scale
+    mt = torch.from_numpy(mask)
+    seen = mask.any(-1)  # [B, H, n_q]
+    safe = mt | torch.from_numpy(~seen)[..., None]  # rows with no key: any mask (discarded)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=safe, scale=scale)
+    ref = ref.permute(0, 2, 1, 3).numpy().reshape(B * n_q, H, d)
+    ref_lse = torch.logsumexp(s.masked_fill(~safe, -math.inf), -1).permute(0, 2, 1).numpy().reshape(B * n_q, H)
+    vis = seen.transpose(0, 2, 1).reshape(B * n_q, H)
+    if vis.all() or not vis.any():
+        raise AssertionError("block-sparse pin: the case must mix rows with and without keys")
+    _close(o[vis], ref[vis], 1e-12, 1e-14, "block-sparse attention vs masked torch sdpa (o)")
+    _close(lse[vis], ref_lse[vis], 1e-12, 1e-14, "block-sparse attention vs masked logsumexp (lse)")
+    if not (np.all(o[~vis] == 0.0) and np.all(np.isneginf(lse[~vis]))):
+        raise AssertionError("block-sparse attention: rows without keys must give o = 0, lse = -inf")
+    # every block listed: plain attention of each batch entry
+    full = [list(range(n_kb))] * (B * H * n_qb)
+    off_f = np.arange(0, n_kb * len(full) + 1, n_kb, dtype=np.int32)
+    idx_f = np.array([e for x in full for e in x], dtype=np.int32)
+    o_f, lse_f = orc.attention_block_sparse(q, k, v, off_f, idx_f, bq, bk, scale)
+    ref_f = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+    _close(o_f, ref_f.permute(0, 2, 1, 3).numpy().reshape(B * n_q, H, d), 1e-12, 1e-14,
+           "block-sparse with every block vs torch sdpa")
+    _close(lse_f, torch.logsumexp(s, -1).permute(0, 2, 1).numpy().reshape(B * n_q, H), 1e-12, 1e-14,
+           "block-sparse with every block: lse")
+    # sampled rows equal the same rows of the full result
+    rows = np.array([0, 5, 40, 73], dtype=np.int64)
+    o_r, lse_r = orc.attention_block_sparse(q, k, v, off, idx, bq, bk, scale, rows=rows)
+    if not (np.array_equal(o_r, o[rows]) and np.array_equal(lse_r, lse[rows])):
+        raise AssertionError("block-sparse attention: sampled rows differ from full rows")
+
+
 ALL_PINS = [
     pin_bf16_rounding,
     pin_rmsnorm,
@@ -514,4 +585,5 @@ ALL_PINS = [
     pin_attention_kv_library,
     pin_merge,
     pin_qkv_projection,
+    pin_attention_block_sparse,
 ]

@@ -42,6 +42,16 @@ MUTANTS = {
     "qkv_k_uses_gamma_q": ("part == 1 ? gamma_k : NULL;", "part == 1 ? gamma_q : NULL;"),
     "qkv_part_offset": ("const int64_t f = part * hd + (int64_t)h * d + i;",
                         "const int64_t f = part * hd + (int64_t)h * d + (i ^ 1);"),
+    "bs_query_block_size": ("const int64_t list = ((int64_t)b * n_heads + h) * n_qb + t / block_q;",
+                            "const int64_t list = ((int64_t)b * n_heads + h) * n_qb + t / block_k;"),
+    "bs_list_order": ("const int64_t list = ((int64_t)b * n_heads + h) * n_qb + t / block_q;",
+                      "const int64_t list = ((int64_t)h * batch + b) * n_qb + t / block_q;"),
+    "bs_key_block_off_by_one": ("if (!seen[j / block_k]) continue;\n                const int64_t kr",
+                                "if (!seen[(j + 1) / block_k]) continue;\n                const int64_t kr"),
+    "bs_key_batch_order": ("const int64_t kr = ((b * n_kv + j) * n_heads + h) * (int64_t)d;",
+                           "const int64_t kr = ((j * batch + b) * n_heads + h) * (int64_t)d;"),
+    "bs_lse_no_max": ("lse[r * n_heads + h] = m + log(z);", "lse[r * n_heads + h] = log(z);"),
+    "bs_scale_dropped": ("s_row[j] = scale * qk;", "s_row[j] = qk;"),
     "bf16_round_half_up": ("nearbyint(ax / quantum)", "floor(ax / quantum + 0.5)"),
     "bf16_subnormal_quantum": ("quantum = ldexp(1.0, -133);", "quantum = ldexp(1.0, -134);"),
     "bf16_mantissa_bits": ("quantum = ldexp(1.0, e - 1 - 7);", "quantum = ldexp(1.0, e - 1 - 8);"),
