@@ -373,6 +373,7 @@ def run_gpu(args):
     peaks, peak_src = load_peaks()
     merge_line = measure_merge(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
     qkv_line = measure_qkv(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
+    sparse_line = measure_sparse(h3, w, dev, stream, max(3, args.steps), peaks, peak_src, att_ms)
     att_tflops = flops / (att_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     pro_bytes = 4.0 * w.total * w.n_heads * w.head_dim * 2 + 12.0 * w.total + w.total + 4 * w.head_dim
@@ -406,6 +407,7 @@ def run_gpu(args):
                 "overlap": "uploads and downloads on two copy streams under the previous/next step's kernels"},
         "roofline_merge": merge_line,
         "roofline_qkv": qkv_line,
+        "roofline_sparse": sparse_line,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks.summary(),
     }
@@ -454,6 +456,67 @@ def measure_merge(h3, w, dev, stream, steps, peaks, peak_src):
             "bytes_per_launch": nbytes, "kernel": "merge_kernel<128>", "peak_source": peak_src,
             "note": "not part of the step: the combine of two partial results over split keys, "
                     "on this workload's output shape"}
+
+
+SPARSE_KEEP = 0.25  # share of the off-diagonal key tiles each query-tile pair keeps
+
+
+def _sparse_lists(w):
+    """The block-sparse pattern measured on a single-sequence workload (its diagonal
+    key tiles plus a seeded quarter of the others per (head, 256-row query block))
+    and the FLOPs it leaves: 4 d x (query rows) x (listed keys) per list."""
+    from video_diffusion_transformer_h3attn_b200 import inputs
+    N, H, d = w.total, w.n_heads, w.head_dim
+    off, idx = inputs.block_lists(1, H, N, N, SPARSE_KEEP, seed=w.seed + 77)
+    n_qp, n_kt = -(-N // 256), -(-N // 128)
+    keys = np.full(n_kt, 128, dtype=np.int64)
+    keys[-1] = N - 128 * (n_kt - 1)
+    rows = np.full(n_qp, 256, dtype=np.int64)
+    rows[-1] = N - 256 * (n_qp - 1)
+    cs = np.concatenate([[0], np.cumsum(keys[idx])])
+    keys_per_list = cs[off[1:]] - cs[off[:-1]]
+    flops = 4.0 * d * float(np.sum(np.tile(rows, H) * keys_per_list))
+    return off, idx, flops
+
+
+def measure_sparse(h3, w, dev, stream, steps, peaks, peak_src, dense_ms):
+    """Block-sparse attention on the workload's sequence with the pattern above,
+    timed on its own after the step measurements (not part of the step);
+    tensor-bound on the FLOPs of the listed tiles."""
+    import torch
+    if len(w.seqlens) != 1:
+        return None
+    off, idx, flops = _sparse_lists(w)
+    N, H, d = w.total, w.n_heads, w.head_dim
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = (bf16(a).view(1, N, H, d) for a in (w.q, w.k, w.v))
+    offt = torch.from_numpy(off).to(dev)
+    idxt = torch.from_numpy(idx).to(dev)
+    o = torch.empty_like(q)
+    for _ in range(3):
+        h3.attention_block_sparse(q, k, v, offt, idxt, o=o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        h3.attention_block_sparse(q, k, v, offt, idxt, o=o)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h3.device_status()
+    ms = e0.elapsed_time(e1) / steps
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    del q, k, v, o
+    return {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+            "ms": ms, "flops_per_launch": flops, "density": flops / w.attention_flops(),
+            "speedup_vs_dense": dense_ms / ms, "kernel": "attn_fwd_kernel<128,false> with key lists",
+            "peak_source": "%s bf16_tflops_sustained" % peak_src,
+            "note": "not part of the step: block-sparse attention over this workload's sequence, "
+                    "diagonal key tiles plus a seeded %.0f%% of the others per 256-row query block"
+                    % (100 * SPARSE_KEEP)}
 
 
 def _qkv_inputs(w, dev):
@@ -554,6 +617,13 @@ def run_kernel_only(args):
         lo = torch.empty_like(la)
         run = lambda: h3.merge(oa, la, ob, lb, o=out.view(shape), lse=lo)
         unit = 3.0 * w.total * w.n_heads * (w.head_dim * 2 + 4) / 1e9
+    elif args.kernel_only == "sparse":
+        off, idx, flops = _sparse_lists(w)
+        shape = (1, w.total, w.n_heads, w.head_dim)
+        offt, idxt = torch.from_numpy(off).cuda(), torch.from_numpy(idx).cuda()
+        run = lambda: h3.attention_block_sparse(q.view(shape), k.view(shape), v.view(shape), offt, idxt,
+                                                o=out.view(shape))
+        unit = flops / 1e12
     elif args.kernel_only == "prologue":
         g = (bf16(w.gamma_q), bf16(w.gamma_k)) if w.gamma_q is not None else (None, None)
         pos = torch.from_numpy(w.pos).cuda() if w.pos is not None else None
@@ -581,7 +651,8 @@ def run_kernel_only(args):
     ms = e0.elapsed_time(e1) / args.steps
     print(json.dumps({"kernel": args.kernel_only, "workload": args.workload, "ms": ms,
                       "rate": unit / (ms * 1e-3),
-                      "rate_unit": "TFLOP/s" if args.kernel_only in ("attention", "qkv") else "GB/s"}), flush=True)
+                      "rate_unit": "TFLOP/s" if args.kernel_only in ("attention", "qkv", "sparse") else "GB/s"}),
+          flush=True)
     return 0
 
 
@@ -594,7 +665,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload for --kernel-only runs (tiny, small, joint, 2k, ragged)")
-    ap.add_argument("--kernel-only", choices=["attention", "prologue", "merge", "qkv"],
+    ap.add_argument("--kernel-only", choices=["attention", "prologue", "merge", "qkv", "sparse"],
                     help="launch only this kernel W + K times (profiling runs)")
     args = ap.parse_args()
     if args.kernel_only:

@@ -189,6 +189,41 @@ h3attn_status h3attn_fwd_kv(const void* q, const void* k, const void* v, void* o
                             float softmax_scale, float* lse, void* stream);
 
 /*
+ * h3attn_fwd_block_sparse -- h3attn_fwd_kv in which each group of 256 query rows
+ * attends only to listed blocks of 128 keys.
+ *
+ * The refine-stage timing table of "Open-H3-Regenerate-2K" gains its largest
+ * step from a sparse attention backend ("+ Sol-Attn sparse attention"), and "H3
+ * Runtime Current State" (Next Work) keeps such backends quality-gated; the pages
+ * give no rule for choosing the blocks.  This call executes a given pattern: the
+ * choice of blocks is the caller's.
+ *
+ * Query rows of a sequence form pairs of 128-row tiles, QP = ceil(seqlen_q / 256)
+ * of them; keys form tiles of 128, KT = ceil(seqlen_kv / 128) of them.  List
+ *   c = (b * n_heads + h) * QP + qp
+ * is blk_idx[blk_off[c] .. blk_off[c + 1]): the key tiles that query rows
+ * [256 qp, 256 qp + 256) of batch entry b, head h see.  Each row attends exactly
+ * to the keys of its listed tiles (the last tile holds seqlen_kv - 128 (KT - 1)
+ * keys); arithmetic and rounding are those of h3attn_fwd on that key set; an
+ * empty list is the empty sum, O = 0 and LSE = -inf.
+ *
+ * blk_off: DEVICE int32 [batch * n_heads * QP + 1], non-decreasing, blk_off[0] = 0.
+ * blk_idx: DEVICE int32, each list strictly ascending with entries in [0, KT).
+ *   Both 4-byte aligned; neither is read on the host.  A list whose entries break
+ *   these rules is detected by the kernel: the query rows it serves are not
+ *   written, every other list is processed, and the next h3attn_device_status()
+ *   returns H3ATTN_ERR_INVALID_ARG.  The offsets themselves are trusted: blk_off
+ *   must have the stated length and its entries must lie in [0, entries of blk_idx].
+ * Other arguments, layouts and rules as h3attn_fwd_kv.
+ */
+h3attn_status h3attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, int32_t batch,
+                                      int64_t seqlen_q, int64_t seqlen_kv, int32_t n_heads, int32_t head_dim,
+                                      const int64_t q_strides[3], const int64_t k_strides[3],
+                                      const int64_t v_strides[3], const int64_t o_strides[3],
+                                      const int32_t* blk_off, const int32_t* blk_idx, float softmax_scale,
+                                      float* lse, void* stream);
+
+/*
  * h3attn_merge -- combine two partial results of the same query rows over
  * disjoint key sets:
  *   L = log(exp(lse_a) + exp(lse_b))  (formed as M + log(sum exp(lse_p - M)),

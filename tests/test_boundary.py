@@ -21,7 +21,7 @@ def test_exports_every_declared_symbol(lib):
     names = h3.declared_symbols()
     assert set(names) >= {"h3attn_prologue", "h3attn_fwd", "h3attn_fwd_varlen", "h3attn_version",
                           "h3attn_status_string", "h3attn_last_error", "h3attn_device_status",
-                          "h3attn_fwd_kv", "h3attn_merge"}
+                          "h3attn_fwd_kv", "h3attn_merge", "h3attn_fwd_block_sparse", "h3attn_qkv_fused"}
     for n in names:
         assert hasattr(lib, n), "library does not export %s" % n
 
@@ -88,6 +88,22 @@ def test_fwd_kv_rejects_bad_arguments(lib):
     assert fwd_kv(lib, d=32) == UNSUPPORTED
     assert fwd_kv(lib, Nk=(1 << 30) + 1) == UNSUPPORTED
     assert fwd_kv(lib, strides=(256 * 256, 252, 128)) == MISALIGNED
+
+
+def fwd_sparse(lib, Nq=256, Nk=100, d=128, off=FAKE, idx=FAKE, k=FAKE):
+    s = S3(256 * 256, 256, 128)
+    return lib.h3attn_fwd_block_sparse(FAKE, k, FAKE, FAKE, 1, Nq, Nk, 2, d, s, s, s, s, off, idx, 0.0, None,
+                                       None)
+
+
+def test_fwd_block_sparse_rejects_bad_arguments(lib):
+    assert fwd_sparse(lib, off=None) == INVALID
+    assert fwd_sparse(lib, idx=None) == INVALID
+    assert fwd_sparse(lib, off=FAKE + 2) == MISALIGNED
+    assert fwd_sparse(lib, idx=FAKE + 6) == MISALIGNED
+    assert fwd_sparse(lib, Nq=0) == INVALID
+    assert fwd_sparse(lib, k=None) == INVALID
+    assert fwd_sparse(lib, d=32) == UNSUPPORTED
 
 
 def merge(lib, N=100, d=128, la=FAKE, o=FAKE, strides=(256 * 100, 256, 128), H=2):

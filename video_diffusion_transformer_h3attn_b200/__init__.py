@@ -19,8 +19,9 @@ from typing import Optional, Sequence, Tuple
 
 from . import _build
 
-__all__ = ["prologue", "attention", "attention_varlen", "device_status", "library", "H3AttnError",
-           "KIND_NONE", "KIND_3D", "KIND_1D", "declared_symbols"]
+__all__ = ["prologue", "attention", "attention_varlen", "attention_kv", "attention_block_sparse", "merge",
+           "qkv_fused", "device_status", "library", "H3AttnError", "KIND_NONE", "KIND_3D", "KIND_1D",
+           "declared_symbols"]
 
 KIND_NONE, KIND_3D, KIND_1D = 0, 1, 2
 
@@ -74,6 +75,9 @@ def library() -> ctypes.CDLL:
         lib.h3attn_qkv_fused.restype = ctypes.c_int
         lib.h3attn_qkv_fused.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _I64, _I64_3, _I64_3,
                                          _P, _P, ctypes.c_double, _P, _P, _I32, _I32, _I32, ctypes.c_double, _P]
+        lib.h3attn_fwd_block_sparse.restype = ctypes.c_int
+        lib.h3attn_fwd_block_sparse.argtypes = [_P, _P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64_3, _I64_3,
+                                                _I64_3, _I64_3, _P, _P, ctypes.c_float, _P, _P]
         lib.h3attn_merge.restype = ctypes.c_int
         lib.h3attn_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I64_3, _I64_3,
                                      _I64_3, _P]
@@ -125,7 +129,8 @@ def _ptr(t) -> Optional[int]:
 
 
 def device_status(stream=None, clear: bool = True) -> None:
-    """Synchronise `stream` and raise if a kernel recorded a device-side timeout."""
+    """Synchronise `stream` and raise if a kernel recorded a device-side failure (a
+    timed-out wait, or a block-sparse key list that broke its rules)."""
     _check("h3attn_device_status", library().h3attn_device_status(_stream_handle(stream), int(clear)))
 
 
@@ -265,6 +270,52 @@ def attention_kv(q, k, v, o=None, softmax_scale: Optional[float] = None, return_
     _check("h3attn_fwd_kv", library().h3attn_fwd_kv(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Nq, Nk, H, d, st(q), st(k), st(v), st(o),
         float(softmax_scale or 0.0), _ptr(lse), _stream_handle(stream)))
+    out = o.squeeze(0) if squeeze else o
+    if return_lse:
+        return out, (lse.squeeze(0) if squeeze else lse)
+    return out
+
+
+def attention_block_sparse(q, k, v, blk_off, blk_idx, o=None, softmax_scale: Optional[float] = None,
+                           return_lse: bool = False, stream=None):
+    """Attention in which each group of 256 query rows sees only listed tiles of 128 keys.
+
+    q: bf16 CUDA [B, Nq, H, d] or [Nq, H, d]; k, v: [B, Nk, H, d] or [Nk, H, d].
+    blk_off: int32 CUDA [B*H*ceil(Nq/256) + 1] offsets into blk_idx; list
+    (b*H + h)*ceil(Nq/256) + qp holds the strictly ascending key tiles (of 128 keys)
+    that query rows [256 qp, 256 qp + 256) of (b, h) attend to.  Returns o and, with
+    return_lse, lse fp32 [B, H, Nq]; an empty list gives o = 0 and lse = -inf.  A list
+    that breaks the rules is reported by the next device_status()."""
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16_cuda(name, t)
+    for name, t in (("blk_off", blk_off), ("blk_idx", blk_idx)):
+        if not (t.is_cuda and t.dtype == torch.int32 and t.is_contiguous()):
+            raise TypeError("%s must be a contiguous int32 CUDA tensor" % name)
+    squeeze = q.dim() == 3
+    if squeeze:
+        q, k, v = q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0)
+        if o is not None:
+            o = o.unsqueeze(0)
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q must be [B, Nq, H, d] and k, v one [B, Nk, H, d] shape")
+    B, Nq, H, d = q.shape
+    if k.shape[0] != B or k.shape[2:] != q.shape[2:]:
+        raise ValueError("k, v must match q in batch, heads and head_dim")
+    Nk = k.shape[1]
+    n_lists = B * H * (-(-Nq // 256))
+    if blk_off.numel() != n_lists + 1:
+        raise ValueError("blk_off must have B*H*ceil(Nq/256) + 1 = %d entries" % (n_lists + 1))
+    if blk_idx.numel() == 0:
+        blk_idx = torch.zeros(1, dtype=torch.int32, device=q.device)  # never read: every list is empty
+    if o is None:
+        o = torch.empty((B, Nq, H, d), dtype=q.dtype, device=q.device)
+    _require_bf16_cuda("o", o)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if return_lse else None
+    st = _strides3
+    _check("h3attn_fwd_block_sparse", library().h3attn_fwd_block_sparse(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Nq, Nk, H, d, st(q), st(k), st(v), st(o), _ptr(blk_off),
+        _ptr(blk_idx), float(softmax_scale or 0.0), _ptr(lse), _stream_handle(stream)))
     out = o.squeeze(0) if squeeze else o
     if return_lse:
         return out, (lse.squeeze(0) if squeeze else lse)

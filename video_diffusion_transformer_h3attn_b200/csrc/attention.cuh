@@ -87,6 +87,12 @@ struct AttnParams {
   int64_t seqlen;             // dense: query tokens per sequence
   int64_t seqlen_kv;          // dense: key/value tokens per sequence (may differ, may be 0)
   int64_t total;              // ragged: total tokens (LSE row stride per head)
+  // block-sparse (dense batches; null = every key tile): CSR lists of the key
+  // tiles (kBN keys each) that each (batch, head, query-tile pair) sees, strictly
+  // ascending; list (b * n_heads + h) * n_qpairs + pair
+  const int32_t* blk_off;
+  const int32_t* blk_idx;
+  int64_t n_qpairs;
   float scale_log2;           // softmax_scale * log2(e)
   LaunchCtl ctl;
 };
@@ -191,8 +197,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   const int64_t q_row0 = static_cast<int64_t>(slot_words[3]) * (kQTiles * kBM);
   const int64_t kv_len = kVarlen ? seq_len : p.seqlen_kv;  // keys this sequence's queries see
-  const int nkv = static_cast<int>((kv_len + kBN - 1) / kBN);
-  const int kv_last_valid = static_cast<int>(kv_len - static_cast<int64_t>(nkv - 1) * kBN);
+  int nkv = static_cast<int>((kv_len + kBN - 1) / kBN);
+  int kv_last_valid = static_cast<int>(kv_len - static_cast<int64_t>(nkv - 1) * kBN);
+  // block-sparse: the tile loops below run over the listed key tiles; a list that
+  // is not strictly ascending inside [0, nkv) is reported in the sticky error bits
+  // and its CTA writes nothing (the other CTAs of the launch carry on)
+  const int32_t* kv_list = nullptr;
+  if (!kVarlen && p.blk_off != nullptr) {
+    const int64_t c = (static_cast<int64_t>(batch) * p.n_heads + head) * p.n_qpairs + slot_words[3];
+    const int32_t e0 = __ldg(p.blk_off + c), e1 = __ldg(p.blk_off + c + 1);
+    const int cnt = e1 - e0;
+    kv_list = p.blk_idx + e0;
+    bool bad = cnt < 0 || cnt > nkv;
+    for (int e = threadIdx.x; !bad && e < cnt; e += blockDim.x) {
+      const int32_t x = __ldg(kv_list + e);
+      bad = x < 0 || x >= nkv || (e > 0 && __ldg(kv_list + e - 1) >= x);
+    }
+    if (__syncthreads_or(bad ? 1 : 0)) {
+      if (threadIdx.x == 0) report_error(kErrBadBlockList);
+      return;  // CTA-uniform
+    }
+    if (cnt > 0 && __ldg(kv_list + cnt - 1) != nkv - 1) kv_last_valid = kBN;  // the ragged tile is not listed
+    nkv = cnt;
+  }
   if (nkv == 0) {
     // no keys (a block of a split key set may be empty): the empty sum, O = 0 and
     // LSE = -inf, for the CTA's rows; nothing else runs
@@ -249,6 +276,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                            y_seq + static_cast<int32_t>(q_row0) + t * kBM, head, batch);
       uint32_t it = 0;
       for (int j = 0; j < nkv && ok; ++j) {
+        const int32_t y_kv = y_seq + (kv_list ? __ldg(kv_list + j) : j) * kBN;
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int slot = static_cast<int>(it % kS);
           const uint32_t use = it / kS;
@@ -260,7 +288,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const CUtensorMap* map = kv ? &tm_v : &tm_k;
           for (int a = 0; a < T::kAtoms; ++a)
             ptx::tma_load_4d(sKV + slot * T::kTileBytes + a * T::kAtomBytes, map, bar_kv_full(slot),
-                             a * 64, y_seq + j * kBN, head, batch);
+                             a * 64, y_kv, head, batch);
         }
       }
       if (ok) {

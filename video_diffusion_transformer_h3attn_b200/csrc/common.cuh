@@ -10,7 +10,8 @@ namespace h3 {
 
 // Error bits recorded by kernels in the device error word.
 enum : uint32_t {
-  kErrTimeout = 1u,  // a bounded wait gave up
+  kErrTimeout = 1u,       // a bounded wait gave up
+  kErrBadBlockList = 2u,  // a block-sparse key list was not strictly ascending in range
 };
 
 // Device error word: [0] = sticky error bits, [1] = id of the last launch that
@@ -29,6 +30,9 @@ struct LaunchCtl {
 __device__ __forceinline__ bool launch_failed(const LaunchCtl& ctl) {
   return *reinterpret_cast<volatile uint32_t*>(&g_error_word[1]) == ctl.launch_id;
 }
+
+// An error that leaves the rest of the launch running (no launch id recorded).
+__device__ __forceinline__ void report_error(uint32_t bits) { atomicOr(&g_error_word[0], bits); }
 
 __device__ __forceinline__ void report_failure(const LaunchCtl& ctl, uint32_t bits) {
   atomicOr(&g_error_word[0], bits);

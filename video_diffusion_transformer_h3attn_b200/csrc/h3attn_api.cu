@@ -23,6 +23,13 @@
 
 namespace {
 
+// The projection runs as CTA pairs (M256 tiles across two SMs) unless built
+// with H3_QKV_PAIRS=0.
+#ifndef H3_QKV_PAIRS
+#define H3_QKV_PAIRS 1
+#endif
+constexpr bool kQkvPairs = H3_QKV_PAIRS != 0;
+
 constexpr int kVersion = 10000;  // 1.0.0
 
 thread_local char t_last_error[512] = "";
@@ -179,6 +186,28 @@ int sm_count() {
   return n;
 }
 
+// How many CTA pairs (clusters of two) of a kernel fit on the device at once: the
+// persistent grid of the paired projection.  Falls back to half the SMs.
+int resident_pairs(const void* kernel, int smem_bytes) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2u * static_cast<unsigned>(sm_count()), 1, 1);
+  cfg.blockDim = dim3(h3::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  return n;
+}
+
+h3attn_status fwd_dense(const void* q, const void* k, const void* v, void* o, int32_t batch, int64_t seqlen_q,
+                        int64_t seqlen_kv, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
+                        const int64_t k_strides[3], const int64_t v_strides[3], const int64_t o_strides[3],
+                        float softmax_scale, float* lse, const int32_t* blk_off, const int32_t* blk_idx,
+                        void* stream);
+
 float resolve_scale(float scale, int d) {
   const float s = scale > 0.0f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   return static_cast<float>(static_cast<double>(s) * 1.4426950408889634074);
@@ -216,6 +245,8 @@ int h3attn_device_status(void* stream, int clear) {
     e = cudaMemcpyToSymbol(h3::g_error_word, zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
   }
+  if (word[0] & h3::kErrBadBlockList)
+    return fail(H3ATTN_ERR_INVALID_ARG, "a block-sparse key list was not strictly ascending in range");
   if (word[0] & h3::kErrTimeout)
     return fail(H3ATTN_ERR_DEVICE_TIMEOUT, "a kernel timed out on an internal barrier (launch %u)", word[1]);
   return H3ATTN_OK;
@@ -277,11 +308,39 @@ h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, v
   return H3ATTN_OK;
 }
 
+h3attn_status h3attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, int32_t batch,
+                                      int64_t seqlen_q, int64_t seqlen_kv, int32_t n_heads, int32_t head_dim,
+                                      const int64_t q_strides[3], const int64_t k_strides[3],
+                                      const int64_t v_strides[3], const int64_t o_strides[3],
+                                      const int32_t* blk_off, const int32_t* blk_idx, float softmax_scale,
+                                      float* lse, void* stream) {
+  if (!blk_off || !blk_idx) return fail(H3ATTN_ERR_INVALID_ARG, "null block list");
+  if ((reinterpret_cast<uintptr_t>(blk_off) | reinterpret_cast<uintptr_t>(blk_idx)) & 3u)
+    return fail(H3ATTN_ERR_MISALIGNED, "block lists must be 4-byte aligned");
+  return fwd_dense(q, k, v, o, batch, seqlen_q, seqlen_kv, n_heads, head_dim, q_strides, k_strides, v_strides,
+                   o_strides, softmax_scale, lse, blk_off, blk_idx, stream);
+}
+
 h3attn_status h3attn_fwd_kv(const void* q, const void* k, const void* v, void* o, int32_t batch,
                             int64_t seqlen_q, int64_t seqlen_kv, int32_t n_heads, int32_t head_dim,
                             const int64_t q_strides[3], const int64_t k_strides[3],
                             const int64_t v_strides[3], const int64_t o_strides[3], float softmax_scale,
                             float* lse, void* stream) {
+  return fwd_dense(q, k, v, o, batch, seqlen_q, seqlen_kv, n_heads, head_dim, q_strides, k_strides, v_strides,
+                   o_strides, softmax_scale, lse, nullptr, nullptr, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Dense batches of equal-length sequences (optionally a separate key length and
+// block-sparse key lists): argument checks, tensor maps, launch.
+h3attn_status fwd_dense(const void* q, const void* k, const void* v, void* o, int32_t batch, int64_t seqlen_q,
+                        int64_t seqlen_kv, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
+                        const int64_t k_strides[3], const int64_t v_strides[3], const int64_t o_strides[3],
+                        float softmax_scale, float* lse, const int32_t* blk_off, const int32_t* blk_idx,
+                        void* stream) {
   if (seqlen_kv < 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen_kv must not be negative");
   // with no keys, k and v are never read and may be null (an empty tensor's data pointer)
   const void* k_chk = (seqlen_kv == 0 && !k) ? q : k;
@@ -324,11 +383,18 @@ h3attn_status h3attn_fwd_kv(const void* q, const void* k, const void* v, void* o
   prm.ctl.launch_id = next_launch_id();
 
   const int64_t pairs = (seqlen_q + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM);
+  prm.blk_off = blk_off;
+  prm.blk_idx = blk_idx;
+  prm.n_qpairs = pairs;
   dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return head_dim == 128 ? launch_attention<128, false>(mq, mk, mv, prm, grid, s)
                          : launch_attention<64, false>(mq, mk, mv, prm, grid, s);
 }
+
+}  // namespace
+
+extern "C" {
 
 h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, int32_t batch,
                          int64_t seqlen, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
@@ -477,7 +543,9 @@ h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, v
   const int64_t features = 3 * static_cast<int64_t>(n_heads) * head_dim;
   CUtensorMap mx, mw;
   if ((st = make_map_rows(&mx, x, dim_in, n_tokens, x_tok_stride, h3::kGemmBM)) != H3ATTN_OK) return st;
-  if ((st = make_map_rows(&mw, w, dim_in, features, dim_in, h3::kGemmBN)) != H3ATTN_OK) return st;
+  if ((st = make_map_rows(&mw, w, dim_in, features, dim_in, kQkvPairs ? h3::kGemmBN / 2 : h3::kGemmBN)) !=
+      H3ATTN_OK)
+    return st;
   void* outs[3] = {q_out, k_out, v_out};
   for (int i = 0; i < 3; ++i) {
     prm.out[i] = static_cast<uint16_t*>(outs[i]);
@@ -493,23 +561,28 @@ h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, v
   prm.dim_in = dim_in;
   prm.n_heads = n_heads;
   prm.eps = static_cast<float>(eps);
-  prm.m_tiles = static_cast<int32_t>((n_tokens + h3::kGemmBM - 1) / h3::kGemmBM);
+  const int tile_m = kQkvPairs ? h3::kGemmPairBM : h3::kGemmBM;
+  prm.m_tiles = static_cast<int32_t>((n_tokens + tile_m - 1) / tile_m);
   prm.n_tiles = static_cast<int32_t>(features / h3::kGemmBN);
   if (static_cast<int64_t>(prm.m_tiles) * prm.n_tiles > 0x7FFFFFFF)
     return fail(H3ATTN_ERR_UNSUPPORTED, "too many tiles");
   prm.ctl.launch_id = next_launch_id();
   const int64_t tiles = static_cast<int64_t>(prm.m_tiles) * prm.n_tiles;
-  const unsigned grid = static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (head_dim == 128) {
-    e = ensure_smem_attr(h3::qkv_fused_kernel<128>, h3::QkvTraits::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv)");
-    h3::qkv_fused_kernel<128><<<grid, h3::kGemmThreads, h3::QkvTraits::kSmemBytes, s>>>(mx, mw, prm);
+  if (kQkvPairs) {
+    auto kern = head_dim == 128 ? h3::qkv_fused_pair_kernel<128> : h3::qkv_fused_pair_kernel<64>;
+    e = ensure_smem_attr(kern, h3::QkvPairTraits::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv pair)");
+    const int pairs = resident_pairs(reinterpret_cast<const void*>(kern), h3::QkvPairTraits::kSmemBytes);
+    const unsigned grid = 2u * static_cast<unsigned>(tiles < pairs ? tiles : pairs);
+    kern<<<grid, h3::kGemmThreads, h3::QkvPairTraits::kSmemBytes, s>>>(mx, mw, prm);
   } else {
-    e = ensure_smem_attr(h3::qkv_fused_kernel<64>, h3::QkvTraits::kSmemBytes);
+    const unsigned grid = static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count());
+    auto kern = head_dim == 128 ? h3::qkv_fused_kernel<128> : h3::qkv_fused_kernel<64>;
+    e = ensure_smem_attr(kern, h3::QkvTraits::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv)");
-    h3::qkv_fused_kernel<64><<<grid, h3::kGemmThreads, h3::QkvTraits::kSmemBytes, s>>>(mx, mw, prm);
+    kern<<<grid, h3::kGemmThreads, h3::QkvTraits::kSmemBytes, s>>>(mx, mw, prm);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "qkv launch");

@@ -212,3 +212,38 @@ def sample_rows(total_or_cu, n_rows: int, seed: int, tile: int = 128) -> np.ndar
         rows = sorted(rows[i] for i in keep)
     extra = rng.integers(0, int(cu[-1]), size=max(0, n_rows - len(rows)))
     return np.unique(np.concatenate([np.asarray(rows, dtype=np.int64), extra.astype(np.int64)]))
+
+
+def block_lists(batch: int, n_heads: int, n_q: int, n_kv: int, keep: float, seed: int,
+                q_block: int = 256, k_block: int = 128, diagonal: bool = True,
+                empty_every: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """Seeded block-sparse key lists in CSR form (int32 offsets, int32 indices).
+
+    List c = (b * n_heads + h) * ceil(n_q / q_block) + qb holds, strictly ascending,
+    the key blocks (k_block keys each) that query block qb of (b, h) sees: with
+    ``diagonal``, every key block overlapping rows [qb * q_block, (qb + 1) * q_block)
+    (when such keys exist), plus each other key block independently with
+    probability ``keep`` (one ``random(n_kb)`` draw per list, in list order);
+    ``empty_every`` > 0 empties lists 0, empty_every, 2 * empty_every, ...
+    The pages name a sparse backend but not its pattern: this is a synthetic
+    stand-in of the stated density."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    n_qb = -(-n_q // q_block)
+    n_kb = -(-n_kv // k_block)
+    off = np.zeros(batch * n_heads * n_qb + 1, dtype=np.int64)
+    parts = []
+    for c in range(batch * n_heads * n_qb):
+        sel = rng.random(n_kb) < keep
+        if diagonal:
+            qb = c % n_qb
+            lo = qb * q_block // k_block
+            hi = min(n_kb, -(-min((qb + 1) * q_block, n_q) // k_block))
+            if lo < hi:
+                sel[lo:hi] = True
+        if empty_every and c % empty_every == 0:
+            sel[:] = False
+        t = np.nonzero(sel)[0].astype(np.int32)
+        parts.append(t)
+        off[c + 1] = off[c] + t.size
+    idx = np.concatenate(parts) if parts else np.zeros(0, dtype=np.int32)
+    return off.astype(np.int32), idx.astype(np.int32)
