@@ -581,7 +581,7 @@ def measure_qkv(h3, w, dev, stream, steps, peaks, peak_src):
     del x, wt, bias, out, proj, qp, kp
     return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak, "ms": ms,
             "unfused_ms": ms_unfused, "speedup_vs_unfused": ms_unfused / ms, "flops_per_launch": flops,
-            "kernel": "qkv_fused_kernel<%d>" % d, "peak_source": "%s bf16_tflops (kernel timed alone)" % peak_src,
+            "kernel": "qkv_fused_pair_kernel<%d>" % d, "peak_source": "%s bf16_tflops (kernel timed alone)" % peak_src,
             "note": "not part of the step: projection dim_in = H*d to 3*H*d features with RMSNorm + RoPE in the "
                     "epilogue, on this workload's tokens; unfused = cuBLAS addmm then the prologue kernel"}
 

@@ -33,6 +33,10 @@
 // Tiles are numbered feature-tile fastest, so the CTAs running at once share a
 // few X row blocks and W stays resident in L2 (3*H*d x dim_in bf16 = 57 MB at
 // H*d = dim_in = 3072).  Every barrier wait is bounded (common.cuh).
+//
+// qkv_fused_pair_kernel (below) is the same design on CTA pairs: 256-token tiles
+// whose M256 MMAs span two SMs, each CTA staging half the operands; the host
+// launches it unless the library is built with H3_QKV_PAIRS=0.
 #pragma once
 
 #include <cuda.h>
