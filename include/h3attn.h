@@ -70,11 +70,23 @@ const char* h3attn_last_error(void);
 
 /*
  * Synchronises `stream`, then reads the device error word of the current
- * device: H3ATTN_OK, or H3ATTN_ERR_DEVICE_TIMEOUT if any kernel of this
- * library gave up on a bounded wait since the word was last cleared, or
+ * device: H3ATTN_OK; H3ATTN_ERR_INVALID_ARG if a block-sparse key list broke
+ * its rules (h3attn_fwd_block_sparse); H3ATTN_ERR_DEVICE_TIMEOUT if any kernel
+ * of this library gave up on a bounded wait since the word was last cleared;
  * H3ATTN_ERR_CUDA if the stream reports an error.  clear != 0 resets the word.
  */
 int h3attn_device_status(void* stream, int clear);
+
+/*
+ * h3attn_selftest_wait_timeout -- failure-detection self-test of the bounded
+ * waits every kernel uses.  Enqueues one small kernel that waits on a barrier
+ * nothing will ever complete, with the same bounded wait as the production
+ * kernels: after about one second the wait gives up, records a timeout in the
+ * device error word and the kernel returns (no trap, no fault; the context
+ * stays usable).  The next h3attn_device_status() on `stream` must return
+ * H3ATTN_ERR_DEVICE_TIMEOUT.  Returns H3ATTN_ERR_CUDA if the launch fails.
+ */
+h3attn_status h3attn_selftest_wait_timeout(void* stream);
 
 /*
  * h3attn_prologue -- per-head RMSNorm of Q and K followed by rotary position

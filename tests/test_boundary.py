@@ -21,7 +21,8 @@ def test_exports_every_declared_symbol(lib):
     names = h3.declared_symbols()
     assert set(names) >= {"h3attn_prologue", "h3attn_fwd", "h3attn_fwd_varlen", "h3attn_version",
                           "h3attn_status_string", "h3attn_last_error", "h3attn_device_status",
-                          "h3attn_fwd_kv", "h3attn_merge", "h3attn_fwd_block_sparse", "h3attn_qkv_fused"}
+                          "h3attn_fwd_kv", "h3attn_merge", "h3attn_fwd_block_sparse", "h3attn_qkv_fused",
+                          "h3attn_selftest_wait_timeout"}
     for n in names:
         assert hasattr(lib, n), "library does not export %s" % n
 

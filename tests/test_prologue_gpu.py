@@ -123,3 +123,19 @@ def test_prologue_identity_without_norm_or_rope(h3):
     w = inputs.make_workload("copy", [100], 4, 128, seed=80, norm=False)
     gq, gk = _run(h3, w)
     assert np.array_equal(gq, w.q) and np.array_equal(gk, w.k)
+
+
+@pytest.mark.parametrize("H,d", [(32, 128), (60, 64)])
+def test_prologue_many_heads(h3, orc, H, d):
+    # head counts above the model's (more heads per token than a warp's passes
+    # at the benchmark size); a ragged token count and all three token kinds
+    n = 77
+    w = inputs.make_workload("many%d" % H, [n], H, d, seed=81 + H, norm=True,
+                             sections=(32, 48, 48) if d == 128 else (16, 24, 24))
+    rng = np.random.default_rng(82)
+    w.pos = np.stack([rng.integers(0, 40, n), rng.integers(0, 50, n), rng.integers(0, 90, n)], 1).astype(np.int32)
+    w.kind = rng.integers(0, 3, n).astype(np.uint8)
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "H%d q" % H)
+    check_prologue(gk, rk, "H%d k" % H)

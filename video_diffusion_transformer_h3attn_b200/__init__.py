@@ -20,7 +20,7 @@ from typing import Optional, Sequence, Tuple
 from . import _build
 
 __all__ = ["prologue", "attention", "attention_varlen", "attention_kv", "attention_block_sparse", "merge",
-           "qkv_fused", "device_status", "library", "H3AttnError", "KIND_NONE", "KIND_3D", "KIND_1D",
+           "qkv_fused", "device_status", "selftest_wait_timeout", "library", "H3AttnError", "KIND_NONE", "KIND_3D", "KIND_1D",
            "declared_symbols"]
 
 KIND_NONE, KIND_3D, KIND_1D = 0, 1, 2
@@ -78,6 +78,8 @@ def library() -> ctypes.CDLL:
         lib.h3attn_fwd_block_sparse.restype = ctypes.c_int
         lib.h3attn_fwd_block_sparse.argtypes = [_P, _P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64_3, _I64_3,
                                                 _I64_3, _I64_3, _P, _P, ctypes.c_float, _P, _P]
+        lib.h3attn_selftest_wait_timeout.restype = ctypes.c_int
+        lib.h3attn_selftest_wait_timeout.argtypes = [_P]
         lib.h3attn_merge.restype = ctypes.c_int
         lib.h3attn_merge.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _I64, _I32, _I32, _I64_3, _I64_3,
                                      _I64_3, _P]
@@ -132,6 +134,13 @@ def device_status(stream=None, clear: bool = True) -> None:
     """Synchronise `stream` and raise if a kernel recorded a device-side failure (a
     timed-out wait, or a block-sparse key list that broke its rules)."""
     _check("h3attn_device_status", library().h3attn_device_status(_stream_handle(stream), int(clear)))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the bounded-wait self-test: a kernel whose one wait can never
+    complete gives up after about a second and records a timeout, which the next
+    device_status() raises (and clears)."""
+    _check("h3attn_selftest_wait_timeout", library().h3attn_selftest_wait_timeout(_stream_handle(stream)))
 
 
 def prologue(q, k, q_out=None, k_out=None, gamma_q=None, gamma_k=None, eps: float = 1e-6,

@@ -20,6 +20,7 @@
 #include "merge.cuh"
 #include "prologue.cuh"
 #include "qkv.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -249,6 +250,15 @@ int h3attn_device_status(void* stream, int clear) {
     return fail(H3ATTN_ERR_INVALID_ARG, "a block-sparse key list was not strictly ascending in range");
   if (word[0] & h3::kErrTimeout)
     return fail(H3ATTN_ERR_DEVICE_TIMEOUT, "a kernel timed out on an internal barrier (launch %u)", word[1]);
+  return H3ATTN_OK;
+}
+
+h3attn_status h3attn_selftest_wait_timeout(void* stream) {
+  h3::LaunchCtl ctl;
+  ctl.launch_id = next_launch_id();
+  h3::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ctl);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
   return H3ATTN_OK;
 }
 
