@@ -7,8 +7,9 @@
  * kernel), then non-causal softmax(Q K^T * scale) V over a packed token
  * sequence (one attention kernel, dense or ragged).  Around it: attention
  * against a separate key block and the log-sum-exp merge of such partial
- * results (key-split schedules), and the Q/K/V projection with the prologue
- * fused into its epilogue.
+ * results (key-split schedules), block-sparse attention over given lists of key
+ * tiles, the Q/K/V projection with the prologue fused into its epilogue, and a
+ * self-test of the kernels' bounded waits.
  *
  * Sources of the operations (web pages about the H3 runtimes):
  *   - "H3 Runtime Current State", Owned Performance Kernels: a fused Q/K
