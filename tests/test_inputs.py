@@ -43,3 +43,52 @@ def test_sample_rows_cover_boundaries():
     for r in (0, 299, 300, 699, 127, 128, 427, 428):
         assert r in rows
     assert rows.min() >= 0 and rows.max() < 700
+
+
+def _lists(off, idx):
+    return [idx[off[c]:off[c + 1]] for c in range(len(off) - 1)]
+
+
+def test_block_lists_are_valid_and_seeded():
+    B, H, nq, nk = 2, 3, 700, 900
+    off, idx = inputs.block_lists(B, H, nq, nk, 0.3, seed=5, empty_every=4)
+    n_qb, n_kb = -(-nq // 256), -(-nk // 128)
+    assert off.dtype == np.int32 and idx.dtype == np.int32
+    assert off.shape == (B * H * n_qb + 1,) and off[0] == 0 and off[-1] == idx.size
+    for c, lst in enumerate(_lists(off, idx)):
+        assert np.all(np.diff(lst) > 0) and (lst.size == 0 or (lst[0] >= 0 and lst[-1] < n_kb))
+        qb = c % n_qb
+        if c % 4 == 0:
+            assert lst.size == 0
+        else:  # the key tiles overlapping the query block's own rows are always listed
+            lo, hi = qb * 256 // 128, min(n_kb, -(-min((qb + 1) * 256, nq) // 128))
+            assert set(range(lo, hi)) <= set(lst.tolist())
+    off2, idx2 = inputs.block_lists(B, H, nq, nk, 0.3, seed=5, empty_every=4)
+    assert np.array_equal(off, off2) and np.array_equal(idx, idx2)
+
+
+def test_block_lists_density_follows_keep():
+    off, idx = inputs.block_lists(1, 8, 4096, 65536, 0.25, seed=9, diagonal=False)
+    n_kb = 65536 // 128
+    share = idx.size / ((len(off) - 1) * n_kb)
+    assert abs(share - 0.25) < 0.01
+    off1, idx1 = inputs.block_lists(1, 2, 300, 300, 1.0, seed=1)
+    assert all(len(lst) == 3 for lst in _lists(off1, idx1))  # every tile of 300 keys
+
+
+def test_bench_sparse_flops_match_a_mask_count():
+    """The benchmark's FLOP count of a block-sparse launch equals 4 d x the number
+    of visible (query, key) pairs counted on the dense mask."""
+    import bench
+    w = inputs.make_workload("sp", [1000], 2, 64, seed=3, norm=False)
+    w.seed = 11
+    off, idx, flops = bench._sparse_lists(w)
+    N, H, d = w.total, w.n_heads, w.head_dim
+    n_qp = -(-N // 256)
+    mask = np.zeros((H, N, N), dtype=bool)
+    for h in range(H):
+        for qp in range(n_qp):
+            c = h * n_qp + qp
+            for t in idx[off[c]:off[c + 1]]:
+                mask[h, 256 * qp:256 * (qp + 1), 128 * int(t):128 * (int(t) + 1)] = True
+    assert flops == 4.0 * d * int(mask.sum())
