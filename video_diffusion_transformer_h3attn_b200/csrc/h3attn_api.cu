@@ -203,15 +203,67 @@ int resident_pairs(const void* kernel, int smem_bytes) {
   return n;
 }
 
+float resolve_scale(float scale, int d) {
+  const float s = scale > 0.0f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  return static_cast<float>(static_cast<double>(s) * 1.4426950408889634074);
+}
+
+// Dense batches of equal-length sequences (optionally a separate key length and
+// block-sparse key lists): argument checks, tensor maps, launch.
 h3attn_status fwd_dense(const void* q, const void* k, const void* v, void* o, int32_t batch, int64_t seqlen_q,
                         int64_t seqlen_kv, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
                         const int64_t k_strides[3], const int64_t v_strides[3], const int64_t o_strides[3],
                         float softmax_scale, float* lse, const int32_t* blk_off, const int32_t* blk_idx,
-                        void* stream);
+                        void* stream) {
+  if (seqlen_kv < 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen_kv must not be negative");
+  // with no keys, k and v are never read and may be null (an empty tensor's data pointer)
+  const void* k_chk = (seqlen_kv == 0 && !k) ? q : k;
+  const void* v_chk = (seqlen_kv == 0 && !v) ? q : v;
+  h3attn_status st = check_common(q, k_chk, v_chk, o, n_heads, head_dim);
+  if (st != H3ATTN_OK) return st;
+  if (batch <= 0 || batch > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "batch must be in [1, 65535]");
+  if (seqlen_q <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be positive");
+  if (seqlen_q > (int64_t(1) << 30) || seqlen_kv > (int64_t(1) << 30))
+    return fail(H3ATTN_ERR_UNSUPPORTED, "seqlen too large");
+  if ((st = check_strides(q_strides, 3, "q")) != H3ATTN_OK) return st;
+  if ((st = check_strides(k_strides, 3, "k")) != H3ATTN_OK) return st;
+  if ((st = check_strides(v_strides, 3, "v")) != H3ATTN_OK) return st;
+  if ((st = check_strides(o_strides, 3, "o")) != H3ATTN_OK) return st;
+  if (!std::isfinite(softmax_scale)) return fail(H3ATTN_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(H3ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
 
-float resolve_scale(float scale, int d) {
-  const float s = scale > 0.0f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
-  return static_cast<float>(static_cast<double>(s) * 1.4426950408889634074);
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, head_dim, seqlen_q, n_heads, batch, q_strides[1], q_strides[2], q_strides[0])) != H3ATTN_OK) return st;
+  if (seqlen_kv > 0) {
+    if ((st = make_map(&mk, k, head_dim, seqlen_kv, n_heads, batch, k_strides[1], k_strides[2], k_strides[0])) != H3ATTN_OK) return st;
+    if ((st = make_map(&mv, v, head_dim, seqlen_kv, n_heads, batch, v_strides[1], v_strides[2], v_strides[0])) != H3ATTN_OK) return st;
+  } else {
+    mk = mq;  // no keys: the kernel writes the empty result and reads neither map
+    mv = mq;
+  }
+
+  h3::AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.o = static_cast<uint16_t*>(o);
+  prm.o_batch = o_strides[0];
+  prm.o_tok = o_strides[1];
+  prm.o_head = o_strides[2];
+  prm.lse = lse;
+  prm.n_heads = n_heads;
+  prm.seqlen = seqlen_q;
+  prm.seqlen_kv = seqlen_kv;
+  prm.total = seqlen_q;
+  prm.scale_log2 = resolve_scale(softmax_scale, head_dim);
+  prm.ctl.launch_id = next_launch_id();
+
+  const int64_t pairs = (seqlen_q + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM);
+  prm.blk_off = blk_off;
+  prm.blk_idx = blk_idx;
+  prm.n_qpairs = pairs;
+  dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return head_dim == 128 ? launch_attention<128, false>(mq, mk, mv, prm, grid, s)
+                         : launch_attention<64, false>(mq, mk, mv, prm, grid, s);
 }
 
 }  // namespace
@@ -339,72 +391,6 @@ h3attn_status h3attn_fwd_kv(const void* q, const void* k, const void* v, void* o
   return fwd_dense(q, k, v, o, batch, seqlen_q, seqlen_kv, n_heads, head_dim, q_strides, k_strides, v_strides,
                    o_strides, softmax_scale, lse, nullptr, nullptr, stream);
 }
-
-}  // extern "C"
-
-namespace {
-
-// Dense batches of equal-length sequences (optionally a separate key length and
-// block-sparse key lists): argument checks, tensor maps, launch.
-h3attn_status fwd_dense(const void* q, const void* k, const void* v, void* o, int32_t batch, int64_t seqlen_q,
-                        int64_t seqlen_kv, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
-                        const int64_t k_strides[3], const int64_t v_strides[3], const int64_t o_strides[3],
-                        float softmax_scale, float* lse, const int32_t* blk_off, const int32_t* blk_idx,
-                        void* stream) {
-  if (seqlen_kv < 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen_kv must not be negative");
-  // with no keys, k and v are never read and may be null (an empty tensor's data pointer)
-  const void* k_chk = (seqlen_kv == 0 && !k) ? q : k;
-  const void* v_chk = (seqlen_kv == 0 && !v) ? q : v;
-  h3attn_status st = check_common(q, k_chk, v_chk, o, n_heads, head_dim);
-  if (st != H3ATTN_OK) return st;
-  if (batch <= 0 || batch > 65535) return fail(H3ATTN_ERR_INVALID_ARG, "batch must be in [1, 65535]");
-  if (seqlen_q <= 0) return fail(H3ATTN_ERR_INVALID_ARG, "seqlen must be positive");
-  if (seqlen_q > (int64_t(1) << 30) || seqlen_kv > (int64_t(1) << 30))
-    return fail(H3ATTN_ERR_UNSUPPORTED, "seqlen too large");
-  if ((st = check_strides(q_strides, 3, "q")) != H3ATTN_OK) return st;
-  if ((st = check_strides(k_strides, 3, "k")) != H3ATTN_OK) return st;
-  if ((st = check_strides(v_strides, 3, "v")) != H3ATTN_OK) return st;
-  if ((st = check_strides(o_strides, 3, "o")) != H3ATTN_OK) return st;
-  if (!std::isfinite(softmax_scale)) return fail(H3ATTN_ERR_INVALID_ARG, "softmax_scale must be finite");
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(H3ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
-
-  CUtensorMap mq, mk, mv;
-  if ((st = make_map(&mq, q, head_dim, seqlen_q, n_heads, batch, q_strides[1], q_strides[2], q_strides[0])) != H3ATTN_OK) return st;
-  if (seqlen_kv > 0) {
-    if ((st = make_map(&mk, k, head_dim, seqlen_kv, n_heads, batch, k_strides[1], k_strides[2], k_strides[0])) != H3ATTN_OK) return st;
-    if ((st = make_map(&mv, v, head_dim, seqlen_kv, n_heads, batch, v_strides[1], v_strides[2], v_strides[0])) != H3ATTN_OK) return st;
-  } else {
-    mk = mq;  // no keys: the kernel writes the empty result and reads neither map
-    mv = mq;
-  }
-
-  h3::AttnParams prm;
-  std::memset(&prm, 0, sizeof(prm));
-  prm.o = static_cast<uint16_t*>(o);
-  prm.o_batch = o_strides[0];
-  prm.o_tok = o_strides[1];
-  prm.o_head = o_strides[2];
-  prm.lse = lse;
-  prm.n_heads = n_heads;
-  prm.seqlen = seqlen_q;
-  prm.seqlen_kv = seqlen_kv;
-  prm.total = seqlen_q;
-  prm.scale_log2 = resolve_scale(softmax_scale, head_dim);
-  prm.ctl.launch_id = next_launch_id();
-
-  const int64_t pairs = (seqlen_q + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM);
-  prm.blk_off = blk_off;
-  prm.blk_idx = blk_idx;
-  prm.n_qpairs = pairs;
-  dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), static_cast<unsigned>(batch));
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return head_dim == 128 ? launch_attention<128, false>(mq, mk, mv, prm, grid, s)
-                         : launch_attention<64, false>(mq, mk, mv, prm, grid, s);
-}
-
-}  // namespace
-
-extern "C" {
 
 h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o, int32_t batch,
                          int64_t seqlen, int32_t n_heads, int32_t head_dim, const int64_t q_strides[3],
