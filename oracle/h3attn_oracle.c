@@ -38,6 +38,12 @@
  *             "Ragged Ulysses sequence parallelism", "Sequence-sharded 50-block
  *             execution") needs; the identity that the combined parts equal the
  *             attention over all keys is what pins them.
+ *   Block-sparse: attention restricted to listed blocks of keys per block of
+ *             queries (h3o_attention_block_sparse): the execution of a given
+ *             pattern for the sparse backend of the "Open-H3-Regenerate-2K"
+ *             refine table; the pages give no selection rule, so none is here.
+ *   Projection: the Q/K/V projection followed by the same norm and rotation
+ *             (h3o_qkv_norm_rope), for the prologue fused into its epilogue.
  *
  * Every loop below is the definition written out in double precision, in the
  * order stated, with no blocking, fusion or reordering.
