@@ -77,7 +77,7 @@ __device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, u
 }
 
 // ---------------------------------------------------------------------------------
-// TMA (bulk tensor copies, no multicast)
+// TMA (bulk tensor copies, each into the issuing CTA's own shared memory)
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -220,8 +220,8 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Tile load into this CTA's shared memory whose completed bytes are counted on
-// the barrier at shared::cluster address `bar` (the pair's rank-0 barrier).  No
-// multicast: each CTA loads its own half of the pair's operands.
+// the barrier at shared::cluster address `bar` (the pair's rank-0 barrier).  Each
+// CTA loads its own half of the pair's operands; no copy goes to several CTAs.
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                                  int32_t c0, int32_t c1, int32_t c2, int32_t c3) {
   asm volatile(
