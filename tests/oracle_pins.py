@@ -22,8 +22,9 @@ What pins what:
                   sampled rows equal full rows.
   block-sparse    torch scaled_dot_product_attention in float64 with the
                   boolean mask the block lists describe (built by plain loops);
-                  all blocks listed equals unmasked attention; rows with no
-                  key give the empty sum.
+                  a tiny case by 50-digit mpmath brute force; all blocks
+                  listed equals unmasked attention; rows with no key give the
+                  empty sum.
 """
 from __future__ import annotations
 
@@ -566,6 +567,27 @@ def pin_attention_block_sparse(orc):
            "block-sparse with every block vs torch sdpa")
     _close(lse_f, torch.logsumexp(s, -1).permute(0, 2, 1).numpy().reshape(B * n_q, H), 1e-12, 1e-14,
            "block-sparse with every block: lse")
+    # a tiny case by 50-digit brute force over the visible keys (blocks of 2 queries, 3 keys)
+    qs, ks, vs = q[:1, :5, :1, :4].copy(), k[:1, :7, :1, :4].copy(), v[:1, :7, :1, :4].copy()
+    lists_s = [[2, 0], [], [1, 1, 2]]  # unsorted, empty, repeated
+    off_s = np.array([0, 2, 2, 5], dtype=np.int32)
+    idx_s = np.array([e for x in lists_s for e in x], dtype=np.int32)
+    o_s, lse_s = orc.attention_block_sparse(qs, ks, vs, off_s, idx_s, 2, 3, scale)
+    qv, kv, vv = bf16_value(qs)[0, :, 0], bf16_value(ks)[0, :, 0], bf16_value(vs)[0, :, 0]
+    for t in range(5):
+        keys = sorted({j for b in lists_s[t // 2] for j in range(3 * b, min(3 * b + 3, 7))})
+        if not keys:
+            if not (np.all(o_s[t] == 0.0) and np.isneginf(lse_s[t, 0])):
+                raise AssertionError("block-sparse brute force: row %d has no key" % t)
+            continue
+        sj = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(float(qv[t, i])) * mpmath.mpf(float(kv[j, i]))
+                                              for i in range(4)) for j in keys]
+        e = [mpmath.exp(x) for x in sj]
+        den = mpmath.fsum(e)
+        want = [float(mpmath.fsum(e[n] * mpmath.mpf(float(vv[j, i])) for n, j in enumerate(keys)) / den)
+                for i in range(4)]
+        _close(o_s[t, 0], want, 1e-13, 1e-15, "block-sparse vs mpmath, row %d" % t)
+        _close(lse_s[t, 0], float(mpmath.log(den)), 1e-13, 1e-15, "block-sparse lse vs mpmath, row %d" % t)
     # sampled rows equal the same rows of the full result
     rows = np.array([0, 5, 40, 73], dtype=np.int64)
     o_r, lse_r = orc.attention_block_sparse(q, k, v, off, idx, bq, bk, scale, rows=rows)
