@@ -111,6 +111,12 @@ def test_qkv_fused_model_size_sampled(h3, orc):
     _check(h3, orc, 4096, 3072, 24, 128, seed=9, n_rows=96)
 
 
+def test_qkv_fused_2k_sampled(h3, orc):
+    """The 2K clip's token count (129,024) at the model width, as the benchmark
+    launches it (a persistent grid of CTA pairs over 504 x 36 tiles), sampled rows."""
+    _check(h3, orc, 129024, 3072, 24, 128, seed=10, n_rows=64)
+
+
 def test_qkv_fused_matches_projection_then_prologue(h3):
     """Against the unfused path (cuBLAS projection rounded to bf16, then the
     prologue kernel): the two differ by the projection's bf16 rounding only."""
