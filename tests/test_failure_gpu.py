@@ -3,7 +3,6 @@ complete gives up, the host reads the timeout from the device error word, and
 the context stays usable for the next launch."""
 import time
 
-import numpy as np
 import pytest
 
 import oracle
@@ -23,7 +22,6 @@ def h3():
 
 
 def test_bounded_wait_times_out_and_is_reported(h3):
-    import torch
     h3.device_status()  # start from a clear error word
     t0 = time.perf_counter()
     h3.selftest_wait_timeout()

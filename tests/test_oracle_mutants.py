@@ -5,7 +5,6 @@ wrong sign, index or operand), compiles the copy and runs the pins of
 tests/oracle_pins.py against it.  A mutant that passes every pin would mean the
 pins cannot tell that mistake from the real oracle.
 """
-import os
 
 import pytest
 

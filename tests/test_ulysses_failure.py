@@ -8,7 +8,6 @@ import socket
 import time
 from datetime import timedelta
 
-import numpy as np
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp

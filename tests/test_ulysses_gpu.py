@@ -9,7 +9,6 @@ output equal the one-rank output bit for bit:
   * attention over a subset of the heads gives the same bits as those heads of
     the attention over all heads;
 and the one-rank path of ulysses_attention equals the direct calls."""
-import numpy as np
 import pytest
 
 from h3_testlib import to_cuda_bf16
