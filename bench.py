@@ -10,6 +10,11 @@ rank runs its own clip (weak scaling, no collective on the data path).
 
 --impl reference times the fp64 CPU oracle (the correctness reference of this
 project) on the host cores, on a bounded sample of the same workload.
+
+Besides the step, the line carries rooflines of the kernels timed on their own
+after it (not part of the step): the LSE merge on the clip's output shape, the
+fused Q/K/V projection at model width against cuBLAS + the prologue, and
+block-sparse attention on the clip's sequence with a seeded 25% tile pattern.
 """
 from __future__ import annotations
 

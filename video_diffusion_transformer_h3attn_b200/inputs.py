@@ -15,7 +15,9 @@ Recipe (the same for every workload):
   * token order inside a video clip is row-major over the latent grid
     (t, h, w), so token i has coordinates (i // (H*W), (i // W) % H, i % W);
   * audio tokens follow the video tokens and carry one coordinate 0..n_audio-1;
-  * in a ragged batch every sequence restarts its 1D positions at 0.
+  * in a ragged batch every sequence restarts its 1D positions at 0;
+  * block-sparse key lists (block_lists) come from their own generator:
+    diagonal key tiles plus each other tile with a given probability.
 
 The token grids mimic the packed video+audio sequences of the MiniMax-H3
 runtime ("H3 Runtime Current State", Implemented And Validated: packed
