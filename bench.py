@@ -1,20 +1,25 @@
 """Benchmark of the h3attn hot path on B200: one step = the Q/K RMSNorm + RoPE
-prologue followed by dense non-causal attention, on the 2K-refine workload
-(one clip of a 32 x 48 x 84 latent grid = 129,024 tokens, 24 heads of 128).
+prologue followed by non-causal attention on one clip; by default the 2K-refine
+workload (a 32 x 48 x 84 latent grid = 129,024 tokens, 24 heads of 128).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl h3attn|reference]
+                    [--workload tiny|small|joint|2k|ragged] [--parallel replicas|ulysses]
+    python bench.py --table [names]      one line per workload, with the oracle beside it
 
 Prints one JSON line (rank 0).  Metric: attention forward TFLOP/s counted as
-4 * N^2 * d * H per clip, whole job, max time over ranks.  With N GPUs every
-rank runs its own clip (weak scaling, no collective on the data path).
+4 * N^2 * d * H per clip (summed over the sequences of a ragged batch), whole
+job, max time over ranks.  --parallel replicas (default): every rank runs its
+own clip (weak scaling, no collective on the data path).  --parallel ulysses:
+the ranks share one clip, split by tokens, with NCCL all-to-alls to head shards
+around attention (strong scaling).
 
 --impl reference times the fp64 CPU oracle (the correctness reference of this
 project) on the host cores, on a bounded sample of the same workload.
 
-Besides the step, the line carries rooflines of the kernels timed on their own
-after it (not part of the step): the LSE merge on the clip's output shape, the
-fused Q/K/V projection at model width against cuBLAS + the prologue, and
-block-sparse attention on the clip's sequence with a seeded 25% tile pattern.
+Besides the step, the default line carries rooflines of the kernels timed on
+their own after it (not part of the step): the LSE merge on the clip's output
+shape, the fused Q/K/V projection at model width against cuBLAS + the prologue,
+and block-sparse attention on the clip's sequence with a seeded 25% tile pattern.
 """
 from __future__ import annotations
 
@@ -39,17 +44,33 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def workload_config(w, n_gpus):
-    return {
-        "workload": "2K refine clip: latent grid 32x48x84 = 129024 tokens, 24 heads x 128, "
-                    "Q/K RMSNorm (eps 1e-6) + 3D RoPE 32/48/48 (theta 1e4) + non-causal attention",
-        "global_batch": n_gpus,
+WORKLOAD_TEXT = {
+    "tiny": "tiny clip: 4x8x8 grid = 256 tokens, 2 heads x 64, attention only",
+    "small": "small DiT block: 8x16x24 grid = 3072 tokens, 24 heads x 128, Q/K RMSNorm (eps 1e-6) + 3D RoPE "
+             "32/48/48 (theta 1e4) + non-causal attention",
+    "joint": "joint video+audio clip: 16x30x54 grid = 25920 video + 256 audio = 26176 tokens, 24 heads x 128, "
+             "Q/K RMSNorm + 3D RoPE (video) / 1D RoPE (audio) + non-causal attention",
+    "2k": "2K refine clip: latent grid 32x48x84 = 129024 tokens, 24 heads x 128, Q/K RMSNorm (eps 1e-6) + "
+          "3D RoPE 32/48/48 (theta 1e4) + non-causal attention",
+    "ragged": "ragged packed batch: 4 sequences of 4096/9000/17001/31234 = 61331 tokens, 16 heads x 128, "
+              "1D RoPE (theta 1e4), Q x4, no norm, attention per sequence via cu_seqlens",
+}
+
+
+def workload_config(w, n_gpus, parallel="replicas"):
+    cfg = {
+        "workload": WORKLOAD_TEXT.get(w.name, w.name),
+        "global_batch": n_gpus if parallel == "replicas" else 1,
         "seq_len": int(w.total),
         "heads": int(w.n_heads),
         "head_dim": int(w.head_dim),
-        "parallelism": "replicas" if n_gpus == 1 else "dp%d" % n_gpus,
-        "l2": "inputs larger than L2 (Q, K, V 2.4 GB per clip)",
+        "parallelism": ("replicas" if n_gpus == 1 else "dp%d" % n_gpus) if parallel == "replicas"
+        else "ulysses%d" % n_gpus,
     }
+    qkv_bytes = 3 * w.total * w.n_heads * w.head_dim * 2
+    cfg["l2"] = ("inputs larger than L2 (Q, K, V %.1f GB per clip)" % (qkv_bytes / 1e9) if qkv_bytes > 126e6
+                 else "inputs smaller than L2 (%.1f MB): L2 is not flushed between steps" % (qkv_bytes / 1e6))
+    return cfg
 
 
 def load_peaks():
@@ -122,50 +143,82 @@ def _cores_used():
         return os.cpu_count() or 1
 
 
-def oracle_sample_setup(w, orc):
-    """K' of the whole clip (every query attends to all of it) -- done once."""
+CPU_SAMPLE_PAIRS = 2048   # (query row, head) pairs timed for cpu_baseline
+REFERENCE_STEP_PAIRS = 1024  # (query row, head) pairs per step of --impl reference
+
+
+def oracle_k_prologue(w, orc):
+    """K' of the whole clip (every sampled query attends to all of it): done once, timed."""
     t0 = time.perf_counter()
-    _, k16 = orc.rmsnorm_rope(w.k, w.gamma_k, w.eps, w.pos, w.kind, w.sections, w.theta, want_f64=False)
+    if w.has_prologue:
+        _, k16 = orc.rmsnorm_rope(w.k, w.gamma_k, w.eps, w.pos, w.kind, w.sections, w.theta, want_f64=False)
+    else:
+        k16 = w.k
     return k16, time.perf_counter() - t0
 
 
-def oracle_sample_step(w, orc, k16, rows):
-    """Oracle prologue of the sampled query rows + attention of those rows over all keys."""
-    _, q16 = orc.rmsnorm_rope(w.q[rows], w.gamma_q, w.eps, w.pos[rows], w.kind[rows], w.sections,
-                              w.theta, want_f64=False)
+def sample_pairs(w, n_pairs, seed):
+    """n_pairs (query row, head) pairs: rows that visit every 128-row query tile
+    (inputs.sample_rows_every_tile), heads assigned in turn."""
+    from video_diffusion_transformer_h3attn_b200 import inputs
+    rows = inputs.sample_rows_every_tile(w.cu_seqlens, n_pairs, seed=seed)
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    rows = np.sort(rng.choice(rows, size=min(n_pairs, len(rows)), replace=False))
+    heads = np.arange(len(rows)) % w.n_heads
+    return rows, heads
+
+
+def oracle_pairs(w, orc, k16, rows, heads):
+    """The oracle on the given (row, head) pairs: the prologue of those query rows,
+    then each row's attention over all keys of its sequence, one head per row.
+    Returns the FLOPs of the attention part (4 d per key per pair)."""
+    if w.has_prologue:
+        _, q16 = orc.rmsnorm_rope(w.q[rows], w.gamma_q, w.eps, w.pos[rows], w.kind[rows], w.sections,
+                                  w.theta, want_f64=False)
+    else:
+        q16 = w.q[rows]
     # the oracle reads query rows by index: scatter the sampled rows into a full-size
     # buffer (np.empty maps pages lazily, so only the sampled rows are touched)
-    qbuf = np.empty_like(w.q)
-    qbuf[rows] = q16
-    orc.attention(qbuf, k16, w.v, w.cu_seqlens, rows=rows)
+    flops = 0.0
+    seq_of = np.searchsorted(w.cu_seqlens, rows, side="right") - 1
+    lens = np.diff(w.cu_seqlens)
+    for h in range(w.n_heads):
+        sel = heads == h
+        if not np.any(sel):
+            continue
+        qb = np.empty((w.total, 1, w.head_dim), dtype=np.uint16)
+        qb[rows[sel], 0] = q16[sel, h]
+        orc.attention(qb, np.ascontiguousarray(k16[:, h:h + 1]), np.ascontiguousarray(w.v[:, h:h + 1]),
+                      w.cu_seqlens, rows=rows[sel])
+        flops += 4.0 * w.head_dim * float(np.sum(lens[seq_of[sel]]))
+    return flops
 
 
-def cpu_baseline(w, rows_target_s=15.0):
+def cpu_baseline(w):
+    """The oracle timed on this host: the K prologue of the whole clip, then 2,048
+    (query row, head) pairs over every query tile; extrapolated to the whole clip."""
     import oracle
     orc = oracle.get()
-    k16, t_k = oracle_sample_setup(w, orc)
-    rows = np.arange(4, dtype=np.int64) * 7919 % w.total
+    k16, t_k = oracle_k_prologue(w, orc)
+    rows, heads = sample_pairs(w, CPU_SAMPLE_PAIRS, seed=w.seed + 2000)
     t0 = time.perf_counter()
-    oracle_sample_step(w, orc, k16, rows)
-    t_probe = time.perf_counter() - t0
-    n = int(max(4, min(w.total, len(rows) * rows_target_s / max(t_probe, 1e-3))))
-    rows = np.unique(np.linspace(0, w.total - 1, n).astype(np.int64))
-    t0 = time.perf_counter()
-    oracle_sample_step(w, orc, k16, rows)
-    t_rows = time.perf_counter() - t0
-    flops_rows = 4.0 * len(rows) * w.total * w.head_dim * w.n_heads
-    # whole-clip time: prologue of all Q and K rows (2x the K pass) + attention of every row
-    t_full = 2.0 * t_k + t_rows * w.total / len(rows)
+    flops = oracle_pairs(w, orc, k16, rows, heads)
+    t_pairs = time.perf_counter() - t0
+    # whole clip: the prologue of every Q and K row (twice the K pass) and the
+    # attention of every (row, head) pair at the sampled rate
+    t_full = (2.0 * t_k if w.has_prologue else 0.0) + t_pairs * w.attention_flops() / flops
     return {
         "value": w.attention_flops() / t_full / 1e12,
         "unit": "TFLOP/s",
         "cores": _cores_used(),
         "kind": "oracle",
-        "sample": "%d of %d query rows x %d heads (full keys) + the K prologue of the whole clip; "
-                  "extrapolated linearly to the whole clip (rows are independent and equal cost)"
-                  % (len(rows), w.total, w.n_heads),
-        "sample_tflops": flops_rows / t_rows / 1e12,
-        "seconds": t_k + t_rows,
+        "sample": "%d (query row, head) pairs, rows visiting all %d query tiles of 128, heads in turn, "
+                  "each over every key of its sequence (%s), + the K prologue of the whole clip (%.1f s); "
+                  "extrapolated linearly to the whole clip (pairs are independent, cost proportional to keys)"
+                  % (len(rows), sum(-(-n // 128) for n in w.seqlens),
+                     "%d keys" % w.total if len(w.seqlens) == 1 else "%d sequences" % len(w.seqlens), t_k),
+        "sample_tflops": flops / t_pairs / 1e12,
+        "seconds": t_k + t_pairs,
     }
 
 
@@ -175,30 +228,29 @@ def run_reference(args):
         return 0
     import oracle
     from video_diffusion_transformer_h3attn_b200 import inputs
-    w = inputs.workload(WORKLOAD)
+    w = inputs.workload(args.workload)
     orc = oracle.get()
-    k16, _ = oracle_sample_setup(w, orc)
-    rng = np.random.default_rng(0)
-    n_rows = 8
-    times = []
+    k16, _ = oracle_k_prologue(w, orc)
+    times, flops = [], []
     for i in range(args.warmup + args.steps):
-        rows = np.sort(rng.choice(w.total, n_rows, replace=False)).astype(np.int64)
+        rows, heads = sample_pairs(w, REFERENCE_STEP_PAIRS, seed=w.seed + 3000 + i)
         t0 = time.perf_counter()
-        oracle_sample_step(w, orc, k16, rows)
+        f = oracle_pairs(w, orc, k16, rows, heads)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)
+            flops.append(f)
     step = statistics.mean(times)
-    flops = 4.0 * n_rows * w.total * w.head_dim * w.n_heads
-    value = flops / step / 1e12
+    value = sum(flops) / sum(times) / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores_used(), "kind": "oracle",
-                         "sample": "%d random query rows x %d heads per step (full keys; K prologue "
-                                   "done once before timing)" % (n_rows, w.n_heads)},
+                         "sample": "%d (query row, head) pairs per step, rows visiting every query tile, "
+                                   "each over all keys (the K prologue is done once before timing)"
+                                   % REFERENCE_STEP_PAIRS},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -247,6 +299,91 @@ def reduce_max(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def _bf16(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def host_inputs(w, rows=None):
+    """The workload's inputs (or the token rows `rows` of them) in pinned host memory."""
+    import torch
+    sel = slice(None) if rows is None else rows
+    host = {"q": _bf16(w.q[sel]).pin_memory(), "k": _bf16(w.k[sel]).pin_memory(),
+            "v": _bf16(w.v[sel]).pin_memory()}
+    if w.gamma_q is not None:
+        host["gq"] = _bf16(w.gamma_q).pin_memory()
+        host["gk"] = _bf16(w.gamma_k).pin_memory()
+    if w.pos is not None:
+        host["pos"] = torch.from_numpy(np.ascontiguousarray(w.pos[sel])).pin_memory()
+        host["kind"] = torch.from_numpy(np.ascontiguousarray(w.kind[sel])).pin_memory()
+    if rows is None and len(w.seqlens) > 1:
+        host["cu"] = torch.from_numpy(np.ascontiguousarray(w.cu_seqlens, dtype=np.int32)).pin_memory()
+    return host
+
+
+def step_buffers(w, d):
+    """Q', K' (when the workload has a prologue) and O for one clip on the device."""
+    import torch
+    b = {"o": torch.empty_like(d["q"])}
+    if w.has_prologue:
+        b["qp"] = torch.empty_like(d["q"])
+        b["kp"] = torch.empty_like(d["k"])
+    return b
+
+
+def run_step(h3, w, d, b, ev=None, stream=None):
+    """One pass of the hot path on one clip: the prologue into Q', K' (when the
+    workload has one), then attention (ragged when it packs several sequences).
+    ev = three CUDA events recorded before, between and after the two kernels."""
+    if ev is not None:
+        ev[0].record(stream)
+    if w.has_prologue:
+        h3.prologue(d["q"], d["k"], b["qp"], b["kp"], d.get("gq"), d.get("gk"), w.eps, d.get("pos"),
+                    d.get("kind"), w.sections, w.theta)
+        q, k = b["qp"], b["kp"]
+    else:
+        q, k = d["q"], d["k"]
+    if ev is not None:
+        ev[1].record(stream)
+    if "cu" in d:
+        h3.attention_varlen(q, k, d["v"], d["cu"], w.max_seqlen, b["o"])
+    else:
+        h3.attention(q, k, d["v"], b["o"])
+    if ev is not None:
+        ev[2].record(stream)
+
+
+def prologue_bytes(w):
+    """Algorithmic bytes of one prologue launch: Q and K read and written once, plus
+    positions (12 B) and kind (1 B) per token when RoPE runs, plus both gammas."""
+    b = 4.0 * w.total * w.n_heads * w.head_dim * 2
+    if w.pos is not None:
+        b += 13.0 * w.total
+    if w.gamma_q is not None:
+        b += 4.0 * w.head_dim
+    return b
+
+
+def timed_steps(h3, w, d, b, stream, warmup, steps):
+    """W untimed then K timed steps; returns (ms per step, prologue ms, attention ms)."""
+    import torch
+    for _ in range(warmup):
+        run_step(h3, w, d, b)
+    h3.device_status()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        run_step(h3, w, d, b, evs[i], stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    h3.device_status()
+    pro = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    return t0.elapsed_time(t1) / steps, pro, att
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -264,39 +401,13 @@ def run_gpu(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    w = inputs.workload(WORKLOAD)
+    w = inputs.workload(args.workload)
     dev = torch.device("cuda", local)
-
-    def bf16(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-
-    host = {
-        "q": bf16(w.q).pin_memory(), "k": bf16(w.k).pin_memory(), "v": bf16(w.v).pin_memory(),
-        "gq": bf16(w.gamma_q).pin_memory(), "gk": bf16(w.gamma_k).pin_memory(),
-        "pos": torch.from_numpy(w.pos).pin_memory(), "kind": torch.from_numpy(w.kind).pin_memory(),
-    }
+    host = host_inputs(w)
     d = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
-    qp = torch.empty_like(d["q"])
-    kp = torch.empty_like(d["k"])
-    o = torch.empty_like(d["q"])
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    b = step_buffers(w, d)
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
-
-    ev = {"pro": [], "att": []}
-
-    def step(record=False):
-        if record:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-            e[0].record(stream)
-        h3.prologue(d["q"], d["k"], qp, kp, d["gq"], d["gk"], w.eps, d["pos"], d["kind"], w.sections, w.theta)
-        if record:
-            e[1].record(stream)
-        h3.attention(qp, kp, d["v"], o)
-        if record:
-            e[2].record(stream)
-            ev["pro"].append((e[0], e[1]))
-            ev["att"].append((e[1], e[2]))
 
     def barrier():
         if world > 1:
@@ -307,56 +418,54 @@ def run_gpu(args):
 
     # ---- device-resident timing ----
     for _ in range(args.warmup):
-        step()
+        run_step(h3, w, d, b)
     h3.device_status()
     barrier()
     torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         t0.record(stream)
-        for _ in range(args.steps):
-            step(record=True)
+        for i in range(args.steps):
+            run_step(h3, w, d, b, evs[i], stream)
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
     h3.device_status()
     ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
-    att_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["att"])
-    pro_ms = statistics.mean(a.elapsed_time(b) for a, b in ev["pro"])
+    pro_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
 
     # ---- end to end through the public API: host buffers in, result back to host ----
     # Every step copies its inputs from pinned host memory and its output back.  Two
     # buffer sets and two copy streams let step i+1's upload and step i-1's download
     # run under step i's kernels (the copies use the PCIe engines, the kernels the SMs).
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o.numel() * o.element_size()
-    sets = [dict(d=d, qp=qp, kp=kp, o=o, oh=o_host)]
-    sets.append(dict(d={k: torch.empty_like(v) for k, v in d.items()}, qp=torch.empty_like(qp),
-                     kp=torch.empty_like(kp), o=torch.empty_like(o),
-                     oh=torch.empty(o.shape, dtype=o.dtype).pin_memory()))
+    d2h = b["o"].numel() * b["o"].element_size()
+    sets = [dict(d=d, b=b, oh=torch.empty(b["o"].shape, dtype=b["o"].dtype).pin_memory())]
+    d2 = {k: torch.empty_like(v) for k, v in d.items()}
+    sets.append(dict(d=d2, b=step_buffers(w, d2), oh=torch.empty(b["o"].shape, dtype=b["o"].dtype).pin_memory()))
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("up", "run", "down")}
 
     def e2e_run(n_steps, t_start=None, t_end=None):
         for i in range(n_steps):
-            b = sets[i % 2]
+            st = sets[i % 2]
             e_up, e_run, e_down = ev["up"][i % 2], ev["run"][i % 2], ev["down"][i % 2]
-            s_in.wait_event(e_run)          # set b's previous kernels finished reading it
+            s_in.wait_event(e_run)          # set i%2's previous kernels finished reading it
             if i == 0 and t_start is not None:
                 t_start.record(s_in)
             with torch.cuda.stream(s_in):
                 for k, v in host.items():
-                    b["d"][k].copy_(v, non_blocking=True)
+                    st["d"][k].copy_(v, non_blocking=True)
             e_up.record(s_in)
             stream.wait_event(e_up)
-            stream.wait_event(e_down)       # set b's previous output is already on the host
-            h3.prologue(b["d"]["q"], b["d"]["k"], b["qp"], b["kp"], b["d"]["gq"], b["d"]["gk"], w.eps,
-                        b["d"]["pos"], b["d"]["kind"], w.sections, w.theta)
-            h3.attention(b["qp"], b["kp"], b["d"]["v"], b["o"])
+            stream.wait_event(e_down)       # set i%2's previous output is already on the host
+            run_step(h3, w, st["d"], st["b"])
             e_run.record(stream)
             s_out.wait_event(e_run)
             with torch.cuda.stream(s_out):
-                b["oh"].copy_(b["o"], non_blocking=True)
+                st["oh"].copy_(st["b"]["o"], non_blocking=True)
             e_down.record(s_out)
         if t_end is not None:
             s_out.wait_event(ev["down"][(n_steps - 1) % 2])
@@ -371,17 +480,19 @@ def run_gpu(args):
     barrier()
     h3.device_status()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    del sets, d2
 
     flops = w.attention_flops()
     value = world * flops / (ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
-    merge_line = measure_merge(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
-    qkv_line = measure_qkv(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
-    sparse_line = measure_sparse(h3, w, dev, stream, max(3, args.steps), peaks, peak_src, att_ms)
+    side = {}
+    if not args.no_side and len(w.seqlens) == 1 and w.has_prologue:
+        side["roofline_merge"] = measure_merge(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
+        side["roofline_qkv"] = measure_qkv(h3, w, dev, stream, max(3, args.steps), peaks, peak_src)
+        side["roofline_sparse"] = measure_sparse(h3, w, dev, stream, max(3, args.steps), peaks, peak_src,
+                                                 att_ms)
     att_tflops = flops / (att_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    pro_bytes = 4.0 * w.total * w.n_heads * w.head_dim * 2 + 12.0 * w.total + w.total + 4 * w.head_dim
-    pro_gbs = pro_bytes / (pro_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC,
         "value": value,
@@ -398,23 +509,24 @@ def run_gpu(args):
         "config": workload_config(w, world),
         "pct_of_datasheet_2250": 100.0 * value / world / DATASHEET_BF16_TFLOPS,
         "pct_of_measured_burst": 100.0 * value / world / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
-        "kernels_ms": {"prologue": pro_ms, "attention": att_ms},
+        "kernels_ms": {"prologue": pro_ms if w.has_prologue else 0.0, "attention": att_ms},
         "roofline": {"bound": "tensor", "achieved": att_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": att_tflops / peak, "traffic": profiled_traffic(),
-                     "kernel": "attn_fwd_kernel<128,false>",
+                     "frac": att_tflops / peak,
+                     "traffic": profiled_traffic() if args.workload == WORKLOAD else None,
+                     "kernel": "attn_fwd_kernel<%d,%s>" % (w.head_dim, "true" if "cu" in d else "false"),
                      "peak_source": "%s bf16_tflops_sustained (kernel timed inside a long step)" % peak_src},
-        "roofline_prologue": {"bound": "hbm", "achieved": pro_gbs, "peak": peaks.get("hbm_gbs"),
-                              "unit": "GB/s", "frac": pro_gbs / peaks.get("hbm_gbs", 6650.0),
-                              "peak_source": peak_src},
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "overlap": "uploads and downloads on two copy streams under the previous/next step's kernels"},
-        "roofline_merge": merge_line,
-        "roofline_qkv": qkv_line,
-        "roofline_sparse": sparse_line,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (2 if w.has_prologue else 1) * args.steps,
         "clocks": clocks.summary(),
     }
+    if w.has_prologue:
+        pro_gbs = prologue_bytes(w) / (pro_ms * 1e-3) / 1e9
+        line["roofline_prologue"] = {"bound": "hbm", "achieved": pro_gbs, "peak": peaks.get("hbm_gbs"),
+                                     "unit": "GB/s", "frac": pro_gbs / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+                                     "bytes_per_launch": prologue_bytes(w), "peak_source": peak_src}
+    line.update(side)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
             line["cpu_baseline"] = cpu_baseline(w)
@@ -425,6 +537,165 @@ def run_gpu(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+    return 0
+
+
+def run_ulysses(args):
+    """Ulysses sequence parallelism over the ranks of this job: every rank holds a
+    contiguous token shard of ONE clip (the first N mod P ranks one token more);
+    per step, the prologue of the shard into per-head-group send blocks, an
+    all-to-all to head shards, attention over all N tokens of H/P heads, and an
+    all-to-all back.  Strong scaling: the clip's FLOPs are shared by all ranks."""
+    import torch
+    import torch.distributed as dist
+
+    import video_diffusion_transformer_h3attn_b200 as h3
+    from video_diffusion_transformer_h3attn_b200 import inputs, ulysses
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    args.gpus = world
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    w = inputs.workload(args.workload)
+    dev = torch.device("cuda", local)
+    N, H, dd = w.total, w.n_heads, w.head_dim
+    sizes = [N // world + (1 if r < N % world else 0) for r in range(world)]
+    lo = sum(sizes[:rank])
+    host = host_inputs(w, rows=slice(lo, lo + sizes[rank]))
+    d = {k: v.to(dev) for k, v in host.items()}
+    cu = None
+    if len(w.seqlens) > 1:
+        cu = torch.from_numpy(np.ascontiguousarray(w.cu_seqlens, dtype=np.int32)).to(dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return ulysses.ulysses_attention(d["q"], d["k"], d["v"], sizes, gamma_q=d.get("gq"), gamma_k=d.get("gk"),
+                                         eps=w.eps, pos=d.get("pos"), kind=d.get("kind"), sections=w.sections,
+                                         theta=w.theta, cu_seqlens=cu, max_seqlen=w.max_seqlen)
+
+    for _ in range(args.warmup):
+        step()
+    h3.device_status()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    h3.device_status()
+    ms = reduce_max(t0.elapsed_time(t1) / args.steps, world, dev)
+    flops = w.attention_flops()
+    row_bytes = H * dd * 2
+    n_r = sizes[rank]
+    line = {
+        "metric": METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, world, parallel="ulysses"),
+        "all_to_all_bytes_per_rank": {
+            "before_attention": 3 * n_r * row_bytes * (world - 1) // world,
+            "after_attention": n_r * row_bytes * (world - 1) // world,
+            "note": "rank 0's shard; Q', K', V sent to the other ranks' head groups, O returned"},
+        "e2e": None,
+        "gpu_launches": None,
+        "clocks": clocks.summary(),
+        "note": "one clip split over the ranks by tokens; the exchange goes through NCCL all-to-all "
+                "(a copy on one rank)",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+TABLE_WORKLOADS = ("tiny", "small", "joint", "2k", "ragged")
+TABLE_SAMPLED_ROWS = {"2k": 2048}  # the full fp64 oracle of the 2k clip takes hours on a host
+
+
+def run_table(args):
+    """One JSON line per workload: the step's TFLOP/s against the datasheet and the
+    measured peaks, the prologue's GB/s, the error against the fp64 oracle and the
+    oracle's own time on this host's cores (full for every workload but the 2k
+    clip, which is compared and timed on 2,048 query rows x all heads that visit
+    every query tile, then extrapolated)."""
+    import torch
+
+    import oracle
+    import video_diffusion_transformer_h3attn_b200 as h3
+    from video_diffusion_transformer_h3attn_b200 import inputs
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+    orc = oracle.get()
+    names = TABLE_WORKLOADS if args.table == "all" else tuple(args.table.split(","))
+    for name in names:
+        w = inputs.workload(name)
+        host = host_inputs(w)
+        d = {k: v.to(dev) for k, v in host.items()}
+        b = step_buffers(w, d)
+        ms, pro_ms, att_ms = timed_steps(h3, w, d, b, stream, args.warmup, args.steps)
+        run_step(h3, w, d, b)
+        h3.device_status()
+        gpu_o = b["o"].view(torch.int16).cpu().numpy().view(np.uint16)
+        gpu_qp = b["qp"].view(torch.int16).cpu().numpy().view(np.uint16) if w.has_prologue else None
+        gpu_kp = b["kp"].view(torch.int16).cpu().numpy().view(np.uint16) if w.has_prologue else None
+        del d, b
+        torch.cuda.empty_cache()
+
+        t0 = time.perf_counter()
+        (_, q16), (_, k16) = orc.prologue_workload(w)
+        t_pro = time.perf_counter() - t0
+        max_ulp = None
+        if w.has_prologue:
+            def ordered(x):
+                x = x.astype(np.int32)
+                return np.where(x & 0x8000, -(x & 0x7FFF), x & 0x7FFF)
+            max_ulp = int(max(np.abs(ordered(gpu_qp) - ordered(q16)).max(),
+                              np.abs(ordered(gpu_kp) - ordered(k16)).max()))
+        n_rows = TABLE_SAMPLED_ROWS.get(name)
+        rows = None if n_rows is None else inputs.sample_rows_every_tile(w.cu_seqlens, n_rows, seed=w.seed + 1000)
+        t0 = time.perf_counter()
+        ro, _ = orc.attention(q16, k16, w.v, w.cu_seqlens, rows=rows)
+        t_att = time.perf_counter() - t0
+        got = (gpu_o if rows is None else gpu_o[rows]).astype(np.uint32) << 16
+        err = np.abs(got.view(np.float32).astype(np.float64) - ro)
+        frac = 1.0 if rows is None else len(rows) / w.total
+        oracle_s = t_pro + t_att / frac
+        tf = w.attention_flops() / (ms * 1e-3) / 1e12
+        line = {
+            "table": name, "config": workload_config(w, 1), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "tflops": tf,
+            "pct_of_datasheet_2250": 100.0 * tf / DATASHEET_BF16_TFLOPS,
+            "pct_of_measured_burst": 100.0 * tf / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+            "pct_of_measured_sustained": 100.0 * tf / peaks.get("bf16_tflops_sustained",
+                                                                 FALLBACK_PEAKS["bf16_tflops_sustained"]),
+            "attention_ms": att_ms, "attention_tflops": w.attention_flops() / (att_ms * 1e-3) / 1e12,
+            "prologue_ms": pro_ms if w.has_prologue else None,
+            "prologue_gbs": prologue_bytes(w) / (pro_ms * 1e-3) / 1e9 if w.has_prologue else None,
+            "prologue_max_ulp": max_ulp,
+            "max_abs": float(err.max()), "mean_abs": float(err.mean()),
+            "compared": "every output" if rows is None else
+                        "%d query rows x %d heads visiting every query tile" % (len(rows), w.n_heads),
+            "oracle_s": oracle_s,
+            "oracle_kind": "full" if rows is None else
+                           "prologue of the whole clip + attention of the sampled rows, extrapolated",
+            "oracle_tflops": w.attention_flops() / oracle_s / 1e12,
+            "cores": _cores_used(), "peak_source": peak_src,
+        }
+        print(json.dumps(line), flush=True)
     return 0
 
 
@@ -667,8 +938,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["h3attn", "reference"], default="h3attn")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD,
-                    help="workload for --kernel-only runs (tiny, small, joint, 2k, ragged)")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side measurements (merge, fused projection, block-sparse)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=TABLE_WORKLOADS,
+                    help="workload of the step (default: the 2K refine clip)")
+    ap.add_argument("--parallel", choices=["replicas", "ulysses"], default="replicas",
+                    help="replicas: every rank its own clip (weak scaling); ulysses: one clip split "
+                         "over the ranks by tokens, all-to-all to head shards (strong scaling)")
+    ap.add_argument("--table", nargs="?", const="all", default=None,
+                    help="one line per workload (comma-separated names, default all) with the error "
+                         "against the oracle and the oracle's time")
     ap.add_argument("--kernel-only", choices=["attention", "prologue", "merge", "qkv", "sparse"],
                     help="launch only this kernel W + K times (profiling runs)")
     args = ap.parse_args()
@@ -679,6 +958,10 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.table:
+        return run_table(args)
+    if args.parallel == "ulysses":
+        return run_ulysses(args)
     return run_gpu(args)
 
 

@@ -70,11 +70,15 @@ const char* h3attn_status_string(int status);
 const char* h3attn_last_error(void);
 
 /*
- * Synchronises `stream`, then reads the device error word of the current
- * device: H3ATTN_OK; H3ATTN_ERR_INVALID_ARG if a block-sparse key list broke
- * its rules (h3attn_fwd_block_sparse); H3ATTN_ERR_DEVICE_TIMEOUT if any kernel
- * of this library gave up on a bounded wait since the word was last cleared;
- * H3ATTN_ERR_CUDA if the stream reports an error.  clear != 0 resets the word.
+ * Reads the device error word of the current device once the work already on
+ * `stream` has finished, then synchronises `stream`: H3ATTN_OK;
+ * H3ATTN_ERR_INVALID_ARG if a ragged launch's cu_seqlens or a block-sparse key
+ * list broke its rules (h3attn_fwd_varlen, h3attn_fwd_block_sparse);
+ * H3ATTN_ERR_DEVICE_TIMEOUT if any kernel of this library gave up on a bounded
+ * wait since the word was last cleared; H3ATTN_ERR_CUDA if the stream reports
+ * an error.  The word is read and (clear != 0) zeroed by one atomic exchange
+ * on the device, enqueued on `stream`: an error that work on another stream
+ * records meanwhile is not lost but stays for the next call.
  */
 int h3attn_device_status(void* stream, int clear);
 
@@ -92,6 +96,13 @@ h3attn_status h3attn_selftest_wait_timeout(void* stream);
 /*
  * h3attn_prologue -- per-head RMSNorm of Q and K followed by rotary position
  * embedding, rounded once to bfloat16.
+ *
+ * Source: "H3 Runtime Current State", Owned Performance Kernels (fused Q/K
+ * RMSNorm and RoPE listed as missing); "Buyer Questions: Current Evidence
+ * Status", block composition answer (norm/RoPE between the projection and
+ * attention).  The pages give no formula: the textbook RMSNorm and the
+ * interleaved-pair rotary form are used, with the 3D split of the task's
+ * workloads.
  *
  * For every token n < n_tokens and head h < n_heads, on the row x of length
  * head_dim (Q and K alike, each with its own gamma):
@@ -134,6 +145,12 @@ h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, v
  * h3attn_fwd -- dense non-causal attention over `batch` sequences of equal
  * length seqlen:  O = softmax(Q K^T * scale) V  per (sequence, head).
  *
+ * Source: "Open-H3-Regenerate-2K", Forward table (the standard forward runs
+ * dense attention on one B200); "Buyer Questions: Current Evidence Status",
+ * block composition answer (attention is the largest share of the block).
+ * Video and audio tokens of one clip form one sequence with no mask ("H3
+ * Runtime Current State", Implemented And Validated: packed denoising).
+ *
  * q, k, v, o: bf16 [batch][seqlen][n_heads][head_dim]; each has strides
  *   {batch, token, head} in elements (x_strides[0..2]), last dim contiguous.
  * softmax_scale <= 0 selects 1/sqrt(head_dim).
@@ -155,11 +172,20 @@ h3attn_status h3attn_fwd(const void* q, const void* k, const void* v, void* o,
  * along the token dimension: sequence s owns tokens [cu_seqlens[s],
  * cu_seqlens[s+1]) and attends only to its own keys.
  *
+ * Source: "H3 Runtime Current State", Implemented And Validated ("Ragged
+ * Ulysses sequence parallelism": sequences of unequal length packed together).
+ * The kernel takes the sequences longest first (cost grows with the square of
+ * the length).
+ *
  * q, k, v, o: bf16 [total_tokens][n_heads][head_dim], strides {token, head}.
- * cu_seqlens: DEVICE int32 [nseq + 1], cu_seqlens[0] = 0, non-decreasing,
- *   cu_seqlens[nseq] = total_tokens (not checked on the host: it is device
- *   memory; empty sequences are allowed and produce nothing).
- * max_seqlen: host value >= every sequence length (sizes the launch).
+ * cu_seqlens: DEVICE int32 [nseq + 1] with cu_seqlens[0] = 0, non-decreasing,
+ *   no sequence longer than max_seqlen, cu_seqlens[nseq] = total_tokens; empty
+ *   sequences are allowed and produce nothing.  It is device memory, so the
+ *   host does not read it: the kernel checks these rules before it uses any
+ *   bound, and a descriptor that breaks one makes the launch write nothing and
+ *   the next h3attn_device_status() return H3ATTN_ERR_INVALID_ARG.
+ * max_seqlen: host value >= every sequence length; it caps the launch's grid
+ *   at nseq * ceil(max_seqlen / 256) query-tile pairs per head.
  * lse: NULL, or fp32 [n_heads][total_tokens].
  * nseq <= 65535.  Other rules as h3attn_fwd.
  */

@@ -157,3 +157,96 @@ def test_python_binding_refuses_cpu_tensors():
         h3.attention(x, x, x)
     with pytest.raises(TypeError):
         h3.prologue(x, x)
+
+
+# ---- the Python binding's own checks, run on the host with stand-in CUDA tensors ----
+# The binding must refuse an output that is too small (the kernels write every row
+# through its strides) or on another device before anything reaches the library.
+# Meta tensors wrapped to report a CUDA device stand in for device memory; the
+# library is replaced by a stub that fails the test if a call gets through.
+
+def _fake_cuda(torch, *shape, dtype=None, index=0):
+    class _FakeCuda(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+        @property
+        def device(self):
+            return torch.device("cuda", index)
+
+    return torch.Tensor._make_subclass(_FakeCuda, torch.empty(shape, dtype=dtype or torch.bfloat16, device="meta"))
+
+
+@pytest.fixture
+def no_library(monkeypatch):
+    def refuse():
+        raise AssertionError("the call reached the library")
+    monkeypatch.setattr(h3, "library", refuse)
+
+
+def test_binding_rejects_outputs_of_the_wrong_shape(no_library):
+    torch = pytest.importorskip("torch")
+    f = lambda *s, **kw: _fake_cuda(torch, *s, **kw)
+    q = f(1, 300, 4, 128)
+    for bad in (f(1, 200, 4, 128), f(1, 300, 2, 128), f(300, 4, 128), f(2, 300, 4, 128)):
+        with pytest.raises(ValueError, match="o must have shape"):
+            h3.attention(q, q, q, o=bad)
+        with pytest.raises(ValueError, match="o must have shape"):
+            h3.attention_kv(q, f(1, 50, 4, 128), f(1, 50, 4, 128), o=bad)
+    with pytest.raises(ValueError, match="o must have shape"):
+        h3.attention(q[0], q[0], q[0], o=f(299, 4, 128))
+    qv = f(300, 4, 128)
+    cu = f(3, dtype=torch.int32)
+    with pytest.raises(ValueError, match="o must have shape"):
+        h3.attention_varlen(qv, qv, qv, cu, 200, o=f(299, 4, 128))
+    off = f(4 * 2 + 1, dtype=torch.int32)
+    idx = f(10, dtype=torch.int32)
+    with pytest.raises(ValueError, match="o must have shape"):
+        h3.attention_block_sparse(q, q, q, off, idx, o=f(1, 256, 4, 128))
+    lse = f(1, 4, 300, dtype=torch.float32)
+    with pytest.raises(ValueError, match="o must have shape"):
+        h3.merge(q, lse, q, lse, o=f(1, 300, 4, 64))
+    x = f(300, 512)
+    w = f(3 * 2 * 128, 512)
+    with pytest.raises(ValueError, match="q_out must have shape"):
+        h3.qkv_fused(x, w, 2, q_out=f(200, 2, 128))
+    with pytest.raises(ValueError, match="k_out must have shape"):
+        h3.prologue(qv, qv, f(300, 4, 128), f(300, 4, 64))
+
+
+def test_binding_rejects_outputs_on_another_device(no_library):
+    torch = pytest.importorskip("torch")
+    q = _fake_cuda(torch, 1, 300, 4, 128)
+    with pytest.raises(ValueError, match="cuda:1"):
+        h3.attention(q, q, q, o=_fake_cuda(torch, 1, 300, 4, 128, index=1))
+    with pytest.raises(ValueError, match="cuda:1"):
+        h3.attention(q, _fake_cuda(torch, 1, 300, 4, 128, index=1), q)
+
+
+def test_binding_checks_side_inputs_sizes(no_library):
+    torch = pytest.importorskip("torch")
+    f = lambda *s, **kw: _fake_cuda(torch, *s, **kw)
+    qv, out = f(300, 4, 128), f(300, 4, 128)
+    with pytest.raises(ValueError, match="gamma_q"):
+        h3.prologue(qv, qv, out, out, gamma_q=f(64))
+    with pytest.raises(ValueError, match="pos must be"):
+        h3.prologue(qv, qv, out, out, pos=f(299, 3, dtype=torch.int32), kind=f(300, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="pos must be"):
+        h3.prologue(qv, qv, out, out, pos=f(300, 3, dtype=torch.int32), kind=f(299, dtype=torch.uint8))
+    x, w, o3 = f(300, 512), f(3 * 2 * 128, 512), f(300, 2, 128)
+    with pytest.raises(ValueError, match="bias"):
+        h3.qkv_fused(x, w, 2, bias=f(3 * 2 * 128 - 8), q_out=o3, k_out=o3, v_out=o3)
+
+
+def test_binding_normalises_strides_of_size_one_dimensions():
+    """A dimension of extent 1 is never stepped over, so a stride torch reports for
+    it that the library would reject is passed as a valid one; the others as they are."""
+    torch = pytest.importorskip("torch")
+    from video_diffusion_transformer_h3attn_b200 import _strides2, _strides3
+    t = torch.empty(1, 5, 4, 128).as_strided((1, 5, 4, 128), (0, 512, 128, 1))
+    assert list(_strides3(t)) == [8, 512, 128]
+    t = torch.empty(7, 1, 128).as_strided((7, 1, 128), (128, 3, 1))
+    assert list(_strides2(t)) == [128, 8]
+    t = torch.empty(2, 3, 4, 128)
+    assert list(_strides3(t)) == [3 * 4 * 128, 4 * 128, 128]

@@ -8,7 +8,9 @@ output equal the one-rank output bit for bit:
     the whole tensor, sliced;
   * attention over a subset of the heads gives the same bits as those heads of
     the attention over all heads;
-and the one-rank path of ulysses_attention equals the direct calls."""
+and the one-rank path of ulysses_attention matches the fp64 oracle (and equals
+the direct calls bit for bit)."""
+import numpy as np
 import pytest
 
 from h3_testlib import to_cuda_bf16
@@ -66,15 +68,36 @@ def test_head_subset_attention_is_bitwise_identical(h3, world):
     h3.device_status()
 
 
-def test_ulysses_one_rank_equals_direct_calls(h3):
+@pytest.mark.parametrize("seqlens", [None, [700, 1, 1389]])
+def test_ulysses_one_rank_matches_the_oracle(h3, seqlens):
+    """The whole one-rank Ulysses step (prologue into the send blocks, the
+    exchange, attention, the return exchange) against the oracle's prologue and
+    attention of the same inputs, under the benchmark spec's tolerances; and bit for bit
+    the same as the direct calls."""
     import torch
+    import oracle
+    from h3_testlib import bf16_bits_to_f64, check_attention, from_cuda_bf16
     from video_diffusion_transformer_h3attn_b200 import ulysses
     w = _joint_like()
+    n = w.q.shape[0]
+    lens = [n] if seqlens is None else seqlens
+    assert sum(lens) == n
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     q, k, v = to_cuda_bf16(w.q), to_cuda_bf16(w.k), to_cuda_bf16(w.v)
     g = (to_cuda_bf16(w.gamma_q), to_cuda_bf16(w.gamma_k))
     pos, kind = torch.from_numpy(w.pos).cuda(), torch.from_numpy(w.kind).cuda()
-    o = ulysses.ulysses_attention(q, k, v, [q.shape[0]], gamma_q=g[0], gamma_k=g[1], pos=pos, kind=kind)
+    cu_t = None if seqlens is None else torch.from_numpy(cu).cuda()
+    o = ulysses.ulysses_attention(q, k, v, [n], gamma_q=g[0], gamma_k=g[1], pos=pos, kind=kind,
+                                  cu_seqlens=cu_t, max_seqlen=max(lens))
+    h3.device_status()
+    orc = oracle.get()
+    (_, rq), (_, rk) = orc.prologue_workload(w)
+    ro, _ = orc.attention(rq, rk, w.v, cu)
+    check_attention(bf16_bits_to_f64(from_cuda_bf16(o)), ro, "ulysses one rank", strict=True)
     qp, kp = h3.prologue(q, k, gamma_q=g[0], gamma_k=g[1], pos=pos, kind=kind)
-    ref = h3.attention(qp, kp, v)
+    if seqlens is None:
+        ref = h3.attention(qp, kp, v)
+    else:
+        ref = h3.attention_varlen(qp, kp, v, cu_t, max(lens))
     h3.device_status()
     assert torch.equal(o, ref)

@@ -130,6 +130,64 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _same_device(device, **tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError("%s is on %s, the inputs on %s" % (name, t.device, device))
+
+
+def _require_out(name: str, t, shape, device) -> None:
+    """An output the kernels write row by row through its strides: its shape must
+    be exactly the one the call produces (a smaller view would be written past its
+    end) and it must live on the inputs' device."""
+    _require_bf16_cuda(name, t)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    _same_device(device, **{name: t})
+
+
+def _require_rope_inputs(pos, kind, n_tokens: int, device) -> None:
+    torch = _torch()
+    if pos is None:
+        return
+    if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous():
+        raise TypeError("pos must be a contiguous CUDA int32 tensor [n_tokens, 3]")
+    if kind is None or kind.dtype != torch.uint8 or not kind.is_cuda or not kind.is_contiguous():
+        raise TypeError("kind must be a contiguous CUDA uint8 tensor [n_tokens]")
+    if tuple(pos.shape) != (n_tokens, 3) or kind.numel() != n_tokens:
+        raise ValueError("pos must be [%d, 3] and kind [%d]" % (n_tokens, n_tokens))
+    _same_device(device, pos=pos, kind=kind)
+
+
+def _require_gamma(name: str, g, head_dim: int, device) -> None:
+    if g is None:
+        return
+    _require_bf16_cuda(name, g)
+    if g.numel() != head_dim:
+        raise ValueError("%s must hold head_dim = %d values" % (name, head_dim))
+    _same_device(device, **{name: g})
+
+
+def _strides(t, ndim: int):
+    """The first `ndim` strides of t ({batch, token, head} or {token, head}) for the
+    C ABI; a dimension of extent <= 1 is never stepped over, so a stride torch
+    reports for it that the library would reject (0, or not a multiple of 8
+    elements) is passed as 8."""
+    s = [t.stride(i) for i in range(ndim)]
+    for i in range(ndim):
+        if t.shape[i] <= 1 and (s[i] <= 0 or s[i] % 8):
+            s[i] = 8
+    return (_I64_3 if ndim == 3 else _I64_2)(*s)
+
+
+def _strides3(t):
+    return _strides(t, 3)
+
+
+def _strides2(t):
+    return _strides(t, 2)
+
+
 def device_status(stream=None, clear: bool = True) -> None:
     """Synchronise `stream` and raise if a kernel recorded a device-side failure (a
     timed-out wait, or a block-sparse key list that broke its rules)."""
@@ -157,27 +215,24 @@ def prologue(q, k, q_out=None, k_out=None, gamma_q=None, gamma_k=None, eps: floa
     _require_bf16_cuda("k", k)
     if q.dim() != 3 or q.shape != k.shape or q.stride() != k.stride():
         raise ValueError("q and k must be [n_tokens, n_heads, head_dim] with equal shapes and strides")
+    _same_device(q.device, k=k)
     if q_out is None:
         q_out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
     if k_out is None:
         k_out = torch.empty(k.shape, dtype=k.dtype, device=k.device)
-    _require_bf16_cuda("q_out", q_out)
-    _require_bf16_cuda("k_out", k_out)
-    if q_out.shape != q.shape or q_out.stride() != k_out.stride():
-        raise ValueError("q_out and k_out must match q's shape and share strides")
-    for name, g in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
-        if g is not None:
-            _require_bf16_cuda(name, g)
-    if pos is not None:
-        if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous():
-            raise TypeError("pos must be a contiguous CUDA int32 tensor [n_tokens, 3]")
-        if kind is None or kind.dtype != torch.uint8 or not kind.is_cuda or not kind.is_contiguous():
-            raise TypeError("kind must be a contiguous CUDA uint8 tensor [n_tokens]")
+    _require_out("q_out", q_out, q.shape, q.device)
+    _require_out("k_out", k_out, q.shape, q.device)
+    if q_out.stride() != k_out.stride():
+        raise ValueError("q_out and k_out must share strides")
     n, h, d = q.shape
+    _require_gamma("gamma_q", gamma_q, d, q.device)
+    _require_gamma("gamma_k", gamma_k, d, q.device)
+    _require_rope_inputs(pos, kind, n, q.device)
     st, sh, sw = sections
+    si, so = _strides2(q), _strides2(q_out)
     _check("h3attn_prologue", library().h3attn_prologue(
-        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), n, h, d, q.stride(0), q.stride(1),
-        q_out.stride(0), q_out.stride(1), _ptr(gamma_q), _ptr(gamma_k), float(eps), _ptr(pos),
+        _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), n, h, d, si[0], si[1],
+        so[0], so[1], _ptr(gamma_q), _ptr(gamma_k), float(eps), _ptr(pos),
         _ptr(kind), st, sh, sw, float(theta), _stream_handle(stream)))
     return q_out, k_out
 
@@ -199,12 +254,13 @@ def attention(q, k, v, o=None, softmax_scale: Optional[float] = None, return_lse
             o = o.unsqueeze(0)
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must share a [B, N, H, d] shape")
+    _same_device(q.device, k=k, v=v)
     B, N, H, d = q.shape
     if o is None:
         o = torch.empty((B, N, H, d), dtype=q.dtype, device=q.device)
-    _require_bf16_cuda("o", o)
+    _require_out("o", o, (B, N, H, d), q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if return_lse else None
-    st = lambda t: _I64_3(t.stride(0), t.stride(1), t.stride(2))
+    st = _strides3
     _check("h3attn_fwd", library().h3attn_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, N, H, d, st(q), st(k), st(v), st(o),
         float(softmax_scale or 0.0), _ptr(lse), _stream_handle(stream)))
@@ -227,27 +283,18 @@ def attention_varlen(q, k, v, cu_seqlens, max_seqlen: int, o=None,
         raise ValueError("q, k, v must share a [total, H, d] shape")
     if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or not cu_seqlens.is_contiguous():
         raise TypeError("cu_seqlens must be a contiguous CUDA int32 tensor")
+    _same_device(q.device, k=k, v=v, cu_seqlens=cu_seqlens)
     total, H, d = q.shape
     if o is None:
         o = torch.empty((total, H, d), dtype=q.dtype, device=q.device)
-    _require_bf16_cuda("o", o)
+    _require_out("o", o, (total, H, d), q.device)
     lse = torch.empty((H, total), dtype=torch.float32, device=q.device) if return_lse else None
-    st = lambda t: _I64_2(t.stride(0), t.stride(1))
+    st = _strides2
     _check("h3attn_fwd_varlen", library().h3attn_fwd_varlen(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(cu_seqlens), cu_seqlens.numel() - 1, total,
         int(max_seqlen), H, d, st(q), st(k), st(v), st(o), float(softmax_scale or 0.0), _ptr(lse),
         _stream_handle(stream)))
     return (o, lse) if return_lse else o
-
-
-def _strides3(t):
-    """{batch, token, head} strides; a dimension of extent <= 1 is never stepped
-    over, so its stride (which torch may report as 0) is passed as a valid value."""
-    s = [t.stride(0), t.stride(1), t.stride(2)]
-    for i in range(3):
-        if t.shape[i] <= 1 and (s[i] <= 0 or s[i] % 8):
-            s[i] = 8
-    return _I64_3(*s)
 
 
 def attention_kv(q, k, v, o=None, softmax_scale: Optional[float] = None, return_lse: bool = False,
@@ -271,9 +318,10 @@ def attention_kv(q, k, v, o=None, softmax_scale: Optional[float] = None, return_
     if k.shape[0] != B or k.shape[2:] != q.shape[2:]:
         raise ValueError("k, v must match q in batch, heads and head_dim")
     Nk = k.shape[1]
+    _same_device(q.device, k=k, v=v)
     if o is None:
         o = torch.empty((B, Nq, H, d), dtype=q.dtype, device=q.device)
-    _require_bf16_cuda("o", o)
+    _require_out("o", o, (B, Nq, H, d), q.device)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if return_lse else None
     st = _strides3
     _check("h3attn_fwd_kv", library().h3attn_fwd_kv(
@@ -315,11 +363,12 @@ def attention_block_sparse(q, k, v, blk_off, blk_idx, o=None, softmax_scale: Opt
     n_lists = B * H * (-(-Nq // 256))
     if blk_off.numel() != n_lists + 1:
         raise ValueError("blk_off must have B*H*ceil(Nq/256) + 1 = %d entries" % (n_lists + 1))
+    _same_device(q.device, k=k, v=v, blk_off=blk_off, blk_idx=blk_idx)
     if blk_idx.numel() == 0:
         blk_idx = torch.zeros(1, dtype=torch.int32, device=q.device)  # never read: every list is empty
     if o is None:
         o = torch.empty((B, Nq, H, d), dtype=q.dtype, device=q.device)
-    _require_bf16_cuda("o", o)
+    _require_out("o", o, (B, Nq, H, d), q.device)
     lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if return_lse else None
     st = _strides3
     _check("h3attn_fwd_block_sparse", library().h3attn_fwd_block_sparse(
@@ -352,13 +401,15 @@ def merge(o_a, lse_a, o_b, lse_b, o=None, lse=None, stream=None):
     for name, t in (("lse_a", lse_a), ("lse_b", lse_b)):
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N):
             raise TypeError("%s must be a contiguous CUDA float32 [B, H, N] tensor" % name)
+    _same_device(o_a.device, o_b=o_b, lse_a=lse_a, lse_b=lse_b)
     if o is None:
         o = torch.empty((B, N, H, d), dtype=o_a.dtype, device=o_a.device)
+    _require_out("o", o, (B, N, H, d), o_a.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=o_a.device)
-    _require_bf16_cuda("o", o)
     if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, N):
         raise TypeError("lse must be a contiguous float32 [B, H, N] tensor")
+    _same_device(o_a.device, lse=lse)
     st = _strides3
     _check("h3attn_merge", library().h3attn_merge(
         _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o), _ptr(lse), B, N, H, d,
@@ -386,22 +437,21 @@ def qkv_fused(x, w, n_heads: int, bias=None, q_out=None, k_out=None, v_out=None,
     if w.shape[0] % (3 * H):
         raise ValueError("w must have 3 * n_heads * head_dim rows")
     d = w.shape[0] // (3 * H)
+    _same_device(x.device, w=w)
     outs = []
     for name, t in (("q_out", q_out), ("k_out", k_out), ("v_out", v_out)):
         if t is None:
             t = torch.empty((n, H, d), dtype=x.dtype, device=x.device)
-        _require_bf16_cuda(name, t)
-        if t.shape != (n, H, d):
-            raise ValueError("%s must be [n_tokens, H, d]" % name)
+        _require_out(name, t, (n, H, d), x.device)
         outs.append(t)
-    for name, t in (("bias", bias), ("gamma_q", gamma_q), ("gamma_k", gamma_k)):
-        if t is not None:
-            _require_bf16_cuda(name, t)
-    if pos is not None:
-        if pos.dtype != torch.int32 or not pos.is_cuda or not pos.is_contiguous():
-            raise TypeError("pos must be a contiguous CUDA int32 tensor [n_tokens, 3]")
-        if kind is None or kind.dtype != torch.uint8 or not kind.is_cuda or not kind.is_contiguous():
-            raise TypeError("kind must be a contiguous CUDA uint8 tensor [n_tokens]")
+    if bias is not None:
+        _require_bf16_cuda("bias", bias)
+        if bias.numel() != 3 * H * d:
+            raise ValueError("bias must hold 3 * n_heads * head_dim = %d values" % (3 * H * d))
+        _same_device(x.device, bias=bias)
+    _require_gamma("gamma_q", gamma_q, d, x.device)
+    _require_gamma("gamma_k", gamma_k, d, x.device)
+    _require_rope_inputs(pos, kind, n, x.device)
     st, sh, sw = sections
     tok = _I64_3(*(max(t.stride(0), 8) if n <= 1 else t.stride(0) for t in outs))
     hst = _I64_3(*(t.stride(1) for t in outs))

@@ -68,8 +68,8 @@ struct AttnTraits {
   static constexpr int kTileBytes = kAtoms * kAtomBytes;     // one Q, K or V tile
   static constexpr int kStages = (D == 128) ? 4 : 8;         // K/V ring slots
   static constexpr int kTiles = kQTiles + kStages;
-  // barriers: q, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2]
-  static constexpr int kBarriers = 1 + 2 * kStages + 3 * kQTiles;
+  // barriers: q, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int kBarriers = 1 + 2 * kStages + 3 * kQTiles + 1;
   static constexpr int kSmemBytes =
       1024 /*alignment slack*/ + kTiles * kTileBytes + 8 * kBarriers + 16 + 8 * kSortMax;
   static constexpr uint32_t kTmemCols = 512;
@@ -97,15 +97,6 @@ struct AttnParams {
   LaunchCtl ctl;
 };
 
-// Bounded wait that ignores the launch-failed flag (used to drain copies in flight).
-__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = ptx::globaltimer_ns();
-  while (!ptx::mbar_test(bar, parity)) {
-    if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
-  }
-  return true;
-}
-
 template <int D, bool kVarlen, bool kLse>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -126,6 +117,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto bar_s_full = [&](int t) { return bars + 8u * (1 + 2 * kS + t); };
   auto bar_p_full = [&](int t) { return bars + 8u * (1 + 2 * kS + kQTiles + t); };
   auto bar_o_done = [&](int t) { return bars + 8u * (1 + 2 * kS + 2 * kQTiles + t); };
+  const uint32_t bar_drain = bars + 8u * (1 + 2 * kS + 3 * kQTiles);  // MMA lane's exit after a failure
   volatile uint32_t* const slot_words =
       reinterpret_cast<volatile uint32_t*>(base_ptr + T::kTiles * T::kTileBytes + 8 * T::kBarriers);
   // slot_words[0] = tensor-memory base, [1] = work valid, [2] = sequence, [3] = query-pair index,
@@ -134,6 +126,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const LaunchCtl ctl = p.ctl;
+
+  // ---- ragged descriptor check (before anything reads a sequence bound) -------------
+  // cu_seqlens[0] = 0, non-decreasing, no sequence longer than max_seqlen (p.seqlen,
+  // which sized the grid) and cu_seqlens[nseq] = total.  Every CTA reaches the same
+  // verdict; a descriptor that breaks a rule is reported in the sticky error bits
+  // and the launch writes nothing.
+  if (kVarlen) {
+    bool bad = false;
+    for (int i = threadIdx.x; i < p.nseq; i += blockDim.x) {
+      const int64_t a = __ldg(p.cu_seqlens + i), b = __ldg(p.cu_seqlens + i + 1);
+      bad |= b < a || b - a > p.seqlen;
+    }
+    if (threadIdx.x == 0)
+      bad |= __ldg(p.cu_seqlens) != 0 || static_cast<int64_t>(__ldg(p.cu_seqlens + p.nseq)) != p.total;
+    if (__syncthreads_or(bad ? 1 : 0)) {
+      if (threadIdx.x == 0) report_error(kErrBadSeqlens);
+      return;  // CTA-uniform
+    }
+  }
 
   // ---- work decode (CTA-uniform, published through shared memory) ----------------
   // Ragged batches: the query-tile pairs of all sequences are numbered longest
@@ -250,6 +261,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ptx::mbar_init(bar_p_full(t), kSoftmaxWarps / kQTiles);  // one arrival per warp of the tile
       ptx::mbar_init(bar_o_done(t), 1);
     }
+    ptx::mbar_init(bar_drain, 1);
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tm_q);
     ptx::tma_prefetch_desc(&tm_k);
@@ -299,10 +311,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       if (!ok) {
         // failure: let the copies already issued land before the CTA releases its smem
-        mbar_wait_for(bar_q, 0, 20000000ull);
+        mbar_wait_for(bar_q, 0, kDrainLimitNs);
         const uint32_t first = it > static_cast<uint32_t>(kS) ? it - kS : 0u;
         for (uint32_t u = first; u < it; ++u)
-          mbar_wait_for(bar_kv_full(static_cast<int>(u % kS)), (u / kS) & 1u, 20000000ull);
+          mbar_wait_for(bar_kv_full(static_cast<int>(u % kS)), (u / kS) & 1u, kDrainLimitNs);
       }
     } else if (warp == kMmaWarp && lane == 0) {
       // ================================ MMA issuer ==================================
@@ -408,6 +420,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         if (!ok) break;
         if (has_next) ptx::mma_commit(bar_kv_empty(slot_of(uk)));
+      }
+      if (!ok) {
+        // failure: every MMA already issued must finish writing tensor memory
+        // before the teardown frees it (the next CTA on this SM may own it then)
+        ptx::mma_commit(bar_drain);
+        mbar_wait_for(bar_drain, 0, kDrainLimitNs);
       }
     }
   } else {
@@ -640,6 +658,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 
   // ---- teardown: every thread arrives here, then the allocating warp frees TMEM ----
+  if (warp < kSoftmaxWarps) ptx::tmem_wait_st();  // a softmax warp that left early may have stores in flight
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -12,6 +12,7 @@ namespace h3 {
 enum : uint32_t {
   kErrTimeout = 1u,       // a bounded wait gave up
   kErrBadBlockList = 2u,  // a block-sparse key list was not strictly ascending in range
+  kErrBadSeqlens = 4u,    // a ragged launch's cu_seqlens broke its rules (the launch wrote nothing)
 };
 
 // Device error word: [0] = sticky error bits, [1] = id of the last launch that
@@ -19,6 +20,16 @@ enum : uint32_t {
 // launches).  Lives in the library module (the library is one translation
 // unit, so this is its only definition); read by h3attn_device_status().
 __device__ uint32_t g_error_word[2];
+// Where h3attn_device_status() has the error word exchanged for zero on the
+// device, so that no error recorded between a read and a clear is lost.
+__device__ uint32_t g_status_snapshot[2];
+
+__global__ void status_exchange_kernel(int clear) {
+  if (threadIdx.x == 0) {
+    g_status_snapshot[0] = clear ? atomicExch(&g_error_word[0], 0u) : atomicOr(&g_error_word[0], 0u);
+    g_status_snapshot[1] = clear ? atomicExch(&g_error_word[1], 0u) : atomicOr(&g_error_word[1], 0u);
+  }
+}
 
 // Longest a thread waits on one barrier phase before declaring the launch failed.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
@@ -64,5 +75,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const L
   if (ptx::mbar_test(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, ctl);
 }
+
+// Bounded wait that ignores the launch-failed flag (used on the way out of a
+// failed launch, to drain copies and tensor-core operations still in flight).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_test(bar, parity)) {
+    if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// How long a thread leaving a failed launch waits for its own operations in flight.
+constexpr uint64_t kDrainLimitNs = 20000000ull;  // 20 ms
 
 }  // namespace h3

@@ -287,17 +287,25 @@ const char* h3attn_status_string(int status) {
 const char* h3attn_last_error(void) { return t_last_error; }
 
 int h3attn_device_status(void* stream, int clear) {
+  // The word is read and (with clear) zeroed by one atomic exchange on the device,
+  // ordered after the stream's earlier work, so an error another stream records
+  // meanwhile stays in the word for the next call.  The snapshot it is copied
+  // through is shared, so concurrent calls in this process take turns.
+  static std::mutex status_mutex;
+  std::lock_guard<std::mutex> lock(status_mutex);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  h3::status_exchange_kernel<<<1, 32, 0, st>>>(clear ? 1 : 0);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "status exchange launch");
   uint32_t word[2] = {0, 0};
-  e = cudaMemcpyFromSymbol(word, h3::g_error_word, sizeof(word));
+  e = cudaMemcpyFromSymbolAsync(word, h3::g_status_snapshot, sizeof(word), 0, cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
-  if (clear) {
-    const uint32_t zero[2] = {0, 0};
-    e = cudaMemcpyToSymbol(h3::g_error_word, zero, sizeof(zero));
-    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
-  }
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if (word[0] & h3::kErrBadSeqlens)
+    return fail(H3ATTN_ERR_INVALID_ARG,
+                "cu_seqlens broke its rules (cu[0] = 0, non-decreasing, lengths <= max_seqlen, "
+                "cu[nseq] = total_tokens); that launch wrote nothing");
   if (word[0] & h3::kErrBadBlockList)
     return fail(H3ATTN_ERR_INVALID_ARG, "a block-sparse key list was not strictly ascending in range");
   if (word[0] & h3::kErrTimeout)
@@ -487,8 +495,13 @@ h3attn_status h3attn_fwd_varlen(const void* q, const void* k, const void* v, voi
   prm.scale_log2 = resolve_scale(softmax_scale, head_dim);
   prm.ctl.launch_id = next_launch_id();
 
-  // upper bound on query-tile pairs: each sequence wastes at most one partial pair
-  const int64_t pairs = (total_tokens + h3::kQTiles * h3::kBM - 1) / (h3::kQTiles * h3::kBM) + nseq;
+  // upper bound on query-tile pairs: each sequence wastes at most one partial pair, and
+  // none has more than ceil(max_seqlen / 256) (the kernel checks every length against
+  // max_seqlen before it runs)
+  constexpr int64_t kPairRows = h3::kQTiles * h3::kBM;
+  const int64_t pairs_by_total = (total_tokens + kPairRows - 1) / kPairRows + nseq;
+  const int64_t pairs_by_max = static_cast<int64_t>(nseq) * ((max_seqlen + kPairRows - 1) / kPairRows);
+  const int64_t pairs = pairs_by_total < pairs_by_max ? pairs_by_total : pairs_by_max;
   dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(n_heads), 1);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return head_dim == 128 ? launch_attention<128, true>(mq, mk, mv, prm, grid, s)

@@ -86,8 +86,8 @@ struct QkvTraits {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
   static constexpr int kBBytes = kGemmBN * kGemmBK * 2;   // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
-  // barriers: full[S], empty[S], acc_full[2], acc_empty[2]
-  static constexpr int kBarriers = 2 * kGemmStages + 4;
+  // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
+  static constexpr int kBarriers = 2 * kGemmStages + 5;
   // per epilogue warp: a 32-row x 32-column bf16 staging block (2 KB) that turns
   // its thread-per-row results into row-contiguous global stores
   static constexpr int kStageOutBytes = 32 * 32 * 2;
@@ -107,7 +107,7 @@ struct QkvPairTraits {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;        // 16 KB: this CTA's 128 tokens
   static constexpr int kBBytes = (kGemmBN / 2) * kGemmBK * 2;  // 16 KB: this CTA's 128 W rows
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarriers = 2 * kStages + 4;
+  static constexpr int kBarriers = 2 * kStages + 5;
   static constexpr int kStageOutBytes = QkvTraits::kStageOutBytes;
   static constexpr int kSmemBytes =
       1024 + kStages * kStageBytes + 8 * kBarriers + 16 + kGemmEpiWarps * kStageOutBytes;
@@ -282,6 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto bar_empty = [&](int s) { return bars + 8u * (kS + s); };
   auto bar_acc_full = [&](int b) { return bars + 8u * (2 * kS + b); };
   auto bar_acc_empty = [&](int b) { return bars + 8u * (2 * kS + 2 + b); };
+  const uint32_t bar_drain = bars + 8u * (2 * kS + 4);  // MMA lane's exit after a failure
   volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + 8 * T::kBarriers);
   uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + 8 * T::kBarriers + 16;
 
@@ -300,6 +301,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       ptx::mbar_init(bar_acc_full(b), 1);
       ptx::mbar_init(bar_acc_empty(b), kGemmEpiWarps);
     }
+    ptx::mbar_init(bar_drain, 1);
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tm_x);
     ptx::tma_prefetch_desc(&tm_w);
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (uint32_t u = first; u < it; ++u) {
         const uint64_t t0 = ptx::globaltimer_ns();
         while (!ptx::mbar_test(bar_full(static_cast<int>(u % kS)), (u / kS) & 1u)) {
-          if (ptx::globaltimer_ns() - t0 > 20000000ull) break;
+          if (ptx::globaltimer_ns() - t0 > kDrainLimitNs) break;
         }
       }
     }
@@ -375,6 +377,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ptx::mma_commit(bar_empty(s));
         }
         if (ok) ptx::mma_commit(bar_acc_full(buf));
+      }
+      if (!ok) {
+        // failure: every MMA already issued must finish writing tensor memory
+        // before the teardown frees it
+        ptx::mma_commit(bar_drain);
+        mbar_wait_for(bar_drain, 0, kDrainLimitNs);
       }
     }
   } else {
@@ -432,6 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   auto bar_empty = [&](int s) { return bars + 8u * (kS + s); };
   auto bar_acc_full = [&](int b) { return bars + 8u * (2 * kS + b); };
   auto bar_acc_empty = [&](int b) { return bars + 8u * (2 * kS + 2 + b); };
+  const uint32_t bar_drain = bars + 8u * (2 * kS + 4);  // MMA lane's exit after a failure
   volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + 8 * T::kBarriers);
   uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + 8 * T::kBarriers + 16;
 
@@ -452,6 +461,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       ptx::mbar_init(bar_acc_full(b), 1);
       ptx::mbar_init(bar_acc_empty(b), 2 * kGemmEpiWarps);
     }
+    ptx::mbar_init(bar_drain, 1);
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tm_x);
     ptx::tma_prefetch_desc(&tm_w);
@@ -500,7 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (uint32_t u = first; u < it; ++u) {
           const uint64_t t0 = ptx::globaltimer_ns();
           while (!ptx::mbar_test(bar_full(static_cast<int>(u % kS)), (u / kS) & 1u)) {
-            if (ptx::globaltimer_ns() - t0 > 20000000ull) break;
+            if (ptx::globaltimer_ns() - t0 > kDrainLimitNs) break;
           }
         }
       }
@@ -544,6 +554,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // arrival is still on its way to this CTA when it exits
       for (int j = k >= 2 ? k - 2 : 0; j < k && ok; ++j)
         ok = mbar_wait(bar_acc_empty(j & 1), static_cast<uint32_t>(j >> 1) & 1u, ctl);
+      if (!ok) {
+        // failure: every pair MMA already issued must finish writing both CTAs'
+        // tensor memory before the teardown frees it (arrives on rank 0 only)
+        ptx::mma_commit_pair(bar_drain, 0x1);
+        mbar_wait_for(bar_drain, 0, kDrainLimitNs);
+      }
     }
   } else {
     // ================================= epilogue ===================================

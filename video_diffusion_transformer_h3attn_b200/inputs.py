@@ -109,6 +109,10 @@ class Workload:
         return [int(c[i + 1] - c[i]) for i in range(len(c) - 1)]
 
     @property
+    def max_seqlen(self) -> int:
+        return max([1] + self.seqlens)
+
+    @property
     def has_prologue(self) -> bool:
         return self.pos is not None or self.gamma_q is not None
 
@@ -214,6 +218,28 @@ def sample_rows(total_or_cu, n_rows: int, seed: int, tile: int = 128) -> np.ndar
         rows = sorted(rows[i] for i in keep)
     extra = rng.integers(0, int(cu[-1]), size=max(0, n_rows - len(rows)))
     return np.unique(np.concatenate([np.asarray(rows, dtype=np.int64), extra.astype(np.int64)]))
+
+
+def sample_rows_every_tile(total_or_cu, n_rows: int, seed: int, tile: int = 128) -> np.ndarray:
+    """Query rows that visit every 128-row query tile of every sequence: each
+    sequence's first two and last two rows; in every tile one edge row (its first
+    row in even tiles, its last in odd ones) and one random row inside it; then
+    random rows until there are at least ``n_rows``.  Sorted and unique."""
+    cu = np.asarray(total_or_cu if np.ndim(total_or_cu) else [0, int(total_or_cu)], dtype=np.int64)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = set()
+    for s in range(len(cu) - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        for r in (a, a + 1, b - 2, b - 1):
+            if a <= r < b:
+                rows.add(r)
+        for i, t0 in enumerate(range(a, b, tile)):
+            t1 = min(t0 + tile, b)
+            rows.add(t0 if i % 2 == 0 else t1 - 1)
+            rows.add(int(rng.integers(t0, t1)))
+    while len(rows) < min(n_rows, int(cu[-1])):
+        rows.add(int(rng.integers(0, int(cu[-1]))))
+    return np.asarray(sorted(rows), dtype=np.int64)
 
 
 def block_lists(batch: int, n_heads: int, n_q: int, n_kv: int, keep: float, seed: int,

@@ -101,34 +101,33 @@ def ulysses_attention(q, k, v, sizes: Sequence[int], group=None, *, gamma_q=None
     # 1. prologue fused with the pack: send blocks [P][n_r][Hp][d]
     send_q = torch.empty((world, n_r, Hp, d), dtype=dt, device=dev)
     send_k = torch.empty_like(send_q)
-    send_v = torch.empty_like(send_q)
     for p in range(world):
         heads = slice(p * Hp, (p + 1) * Hp)
         if n_r:
             prologue_fn(q[:, heads], k[:, heads], send_q[p], send_k[p], gamma_q, gamma_k, eps, pos,
                         kind, sections, theta)
-        send_v[p].copy_(v[:, heads])
+    if world == 1:
+        # one rank: the shard is the whole sequence and every head is local, so
+        # nothing moves; attention reads the prologue's output and V in place
+        return attention_fn(send_q[0], send_k[0], v, cu_seqlens, max_seqlen, softmax_scale)
+    send_v = torch.empty_like(send_q)
+    for p in range(world):
+        send_v[p].copy_(v[:, p * Hp:(p + 1) * Hp])
 
     # 2. token shards -> head shards: receive [N][Hp][d] in global token order
     recv = [torch.empty((N, Hp, d), dtype=dt, device=dev) for _ in range(3)]
     out_splits = [s * Hp * d for s in sizes]
     in_splits = [n_r * Hp * d] * world
     for src, dst in zip((send_q, send_k, send_v), recv):
-        if world == 1:
-            dst.copy_(src[0])
-        else:
-            dist.all_to_all_single(dst.view(-1), src.view(-1), out_splits, in_splits, group=group)
+        dist.all_to_all_single(dst.view(-1), src.view(-1), out_splits, in_splits, group=group)
 
     # 3. attention over the whole sequence for this rank's heads
     o_heads = attention_fn(recv[0], recv[1], recv[2], cu_seqlens, max_seqlen, softmax_scale)
 
     # 4. head shards -> token shards, then unpack to [n_r][H][d]
     back = torch.empty((world, n_r, Hp, d), dtype=dt, device=dev)
-    if world == 1:
-        back[0].copy_(o_heads)
-    else:
-        dist.all_to_all_single(back.view(-1), o_heads.contiguous().view(-1), in_splits, out_splits,
-                               group=group)
+    dist.all_to_all_single(back.view(-1), o_heads.contiguous().view(-1), in_splits, out_splits,
+                           group=group)
     o = torch.empty((n_r, H, d), dtype=dt, device=dev)
     for p in range(world):
         o[:, p * Hp:(p + 1) * Hp].copy_(back[p])
