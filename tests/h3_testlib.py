@@ -7,9 +7,16 @@ Tolerances (written here once, used by every parity test):
   attention  the error beyond the half-ulp that storing the exact value as bf16
              costs by itself, e = max(0, |o_gpu - o_ref| - ulp_bf16(o_ref)/2), has
              max <= 1e-2 and mean <= 1e-3 (for |o| >= 4 that half ulp alone exceeds
-             1e-2; for rows over a few keys |o| ~ 1 and it dominates the mean);
-             strict=True (the five named workloads) also requires the plain
-             max |o_gpu - o_ref| <= 1e-2 and mean <= 1e-3;
+             1e-2; for rows over a few keys |o| ~ 1 and it averages ~2e-3, above the
+             mean bound, even for the exactly rounded output);
+             strict=True also requires the plain mean |o_gpu - o_ref| <= 1e-3
+             and (unless plain_max=False) the plain max <= 1e-2: used for the five
+             named workloads, the one-rank Ulysses path and every sequence of 64
+             keys or more, where |o| is small enough that the plain bounds are
+             attainable.  The ragged workload (Q x 4: peaked rows that reproduce one
+             value row, |o| up to ~4) keeps the plain mean but not the plain max:
+             there the correctly rounded exact output alone is 0.0078 from the
+             fp64 value, leaving no room for the rounding of the weights;
   lse        |lse_gpu - lse_ref| <= 1e-3 (fp32 output).
 """
 from __future__ import annotations
@@ -62,7 +69,7 @@ def check_prologue(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str) -> dic
 
 
 def check_attention(o_gpu: np.ndarray, o_ref: np.ndarray, what: str, lse_gpu=None, lse_ref=None,
-                    strict: bool = False) -> dict:
+                    strict: bool = False, plain_max=None) -> dict:
     o_gpu = np.asarray(o_gpu, dtype=np.float64)
     err = np.abs(o_gpu - o_ref)
     excess = np.maximum(err - bf16_half_ulp(o_ref), 0.0)
@@ -73,8 +80,9 @@ def check_attention(o_gpu: np.ndarray, o_ref: np.ndarray, what: str, lse_gpu=Non
         what, stats, np.unravel_index(int(np.argmax(excess)), excess.shape))
     assert stats["mean_excess"] <= ATTN_MEAN_ABS, "%s: %s" % (what, stats)
     if strict:
-        assert stats["max_abs"] <= ATTN_MAX_ABS, "%s (strict): %s" % (what, stats)
         assert stats["mean_abs"] <= ATTN_MEAN_ABS, "%s (strict): %s" % (what, stats)
+    if strict if plain_max is None else plain_max:
+        assert stats["max_abs"] <= ATTN_MAX_ABS, "%s (strict): %s" % (what, stats)
     if lse_gpu is not None:
         le = np.abs(np.asarray(lse_gpu, dtype=np.float64) - lse_ref)
         stats["lse_max_abs"] = float(le.max())

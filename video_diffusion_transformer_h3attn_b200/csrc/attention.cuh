@@ -75,6 +75,7 @@ struct AttnTraits {
   static constexpr uint32_t kTmemCols = 512;
   static_assert(256 + kQTiles * D <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert((kTiles * kTileBytes) % 1024 == 0 && (8 * kBarriers) % 16 == 0, "barrier and scratch alignment");
 };
 
 struct AttnParams {

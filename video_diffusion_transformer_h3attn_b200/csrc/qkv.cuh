@@ -86,14 +86,17 @@ struct QkvTraits {
   static constexpr int kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
   static constexpr int kBBytes = kGemmBN * kGemmBK * 2;   // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
-  // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain
+  // barriers: full[S], empty[S], acc_full[2], acc_empty[2], drain; the area is
+  // padded to 16 bytes so the staging blocks after it stay 16-byte aligned
   static constexpr int kBarriers = 2 * kGemmStages + 5;
+  static constexpr int kBarrierBytes = (8 * kBarriers + 15) / 16 * 16;
   // per epilogue warp: a 32-row x 32-column bf16 staging block (2 KB) that turns
   // its thread-per-row results into row-contiguous global stores
   static constexpr int kStageOutBytes = 32 * 32 * 2;
   static constexpr int kSmemBytes =
-      1024 + kGemmStages * kStageBytes + 8 * kBarriers + 16 + kGemmEpiWarps * kStageOutBytes;
+      1024 + kGemmStages * kStageBytes + kBarrierBytes + 16 + kGemmEpiWarps * kStageOutBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert((kGemmStages * kStageBytes + kBarrierBytes + 16) % 16 == 0, "staging blocks 16-byte aligned");
 };
 
 // The CTA-pair variant: a cluster of two CTAs computes a 256-token x 256-feature
@@ -108,10 +111,12 @@ struct QkvPairTraits {
   static constexpr int kBBytes = (kGemmBN / 2) * kGemmBK * 2;  // 16 KB: this CTA's 128 W rows
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarriers = 2 * kStages + 5;
+  static constexpr int kBarrierBytes = (8 * kBarriers + 15) / 16 * 16;
   static constexpr int kStageOutBytes = QkvTraits::kStageOutBytes;
   static constexpr int kSmemBytes =
-      1024 + kStages * kStageBytes + 8 * kBarriers + 16 + kGemmEpiWarps * kStageOutBytes;
+      1024 + kStages * kStageBytes + kBarrierBytes + 16 + kGemmEpiWarps * kStageOutBytes;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert((kStages * kStageBytes + kBarrierBytes + 16) % 16 == 0, "staging blocks 16-byte aligned");
 };
 constexpr int kGemmPairBM = 2 * kGemmBM;  // tokens per pair tile
 
@@ -283,8 +288,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   auto bar_acc_full = [&](int b) { return bars + 8u * (2 * kS + b); };
   auto bar_acc_empty = [&](int b) { return bars + 8u * (2 * kS + 2 + b); };
   const uint32_t bar_drain = bars + 8u * (2 * kS + 4);  // MMA lane's exit after a failure
-  volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + 8 * T::kBarriers);
-  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + 8 * T::kBarriers + 16;
+  volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + T::kBarrierBytes);
+  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + T::kBarrierBytes + 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -441,8 +446,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   auto bar_acc_full = [&](int b) { return bars + 8u * (2 * kS + b); };
   auto bar_acc_empty = [&](int b) { return bars + 8u * (2 * kS + 2 + b); };
   const uint32_t bar_drain = bars + 8u * (2 * kS + 4);  // MMA lane's exit after a failure
-  volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + 8 * T::kBarriers);
-  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + 8 * T::kBarriers + 16;
+  volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + T::kBarrierBytes);
+  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + T::kBarrierBytes + 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
