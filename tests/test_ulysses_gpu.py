@@ -68,7 +68,7 @@ def test_head_subset_attention_is_bitwise_identical(h3, world):
     h3.device_status()
 
 
-@pytest.mark.parametrize("seqlens", [None, [700, 1, 1389]])
+@pytest.mark.parametrize("seqlens", [None, [300, 1, 507]])
 def test_ulysses_one_rank_matches_the_oracle(h3, seqlens):
     """The whole one-rank Ulysses step (prologue into the send blocks, the
     exchange, attention, the return exchange) against the oracle's prologue and
