@@ -556,6 +556,25 @@ h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, v
       H3ATTN_OK)
     return st;
   void* outs[3] = {q_out, k_out, v_out};
+  // the outputs as [tokens][heads][head_dim] tensor maps with 32 x 32 boxes in the
+  // 64-byte swizzle of the epilogue's staging blocks
+  CUtensorMap mo[3];
+  if (kQkvPairs) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(H3ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    for (int i = 0; i < 3; ++i) {
+      cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(n_heads),
+                            static_cast<cuuint64_t>(n_tokens)};
+      cuuint64_t strides[2] = {static_cast<cuuint64_t>(out_head_strides[i]) * 2,
+                               static_cast<cuuint64_t>(out_tok_strides[i]) * 2};
+      cuuint32_t box[3] = {32, 1, 32};
+      cuuint32_t estr[3] = {1, 1, 1};
+      CUresult r = fn(&mo[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, outs[i], dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(H3ATTN_ERR_INVALID_ARG, "output tensor map rejected (%d)", (int)r);
+    }
+  }
   for (int i = 0; i < 3; ++i) {
     prm.out[i] = static_cast<uint16_t*>(outs[i]);
     prm.out_tok[i] = out_tok_strides[i];
@@ -585,7 +604,7 @@ h3attn_status h3attn_qkv_fused(const void* x, const void* w, const void* bias, v
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(qkv pair)");
     const int pairs = resident_pairs(reinterpret_cast<const void*>(kern), h3::QkvPairTraits::kSmemBytes);
     const unsigned grid = 2u * static_cast<unsigned>(tiles < pairs ? tiles : pairs);
-    kern<<<grid, h3::kGemmThreads, h3::QkvPairTraits::kSmemBytes, s>>>(mx, mw, prm);
+    kern<<<grid, h3::kGemmThreads, h3::QkvPairTraits::kSmemBytes, s>>>(mx, mw, mo[0], mo[1], mo[2], prm);
   } else {
     const unsigned grid = static_cast<unsigned>(tiles < sm_count() ? tiles : sm_count());
     auto kern = head_dim == 128 ? h3::qkv_fused_kernel<128> : h3::qkv_fused_kernel<64>;

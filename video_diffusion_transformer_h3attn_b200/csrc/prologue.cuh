@@ -15,12 +15,16 @@
 //
 // Precision: x*gamma is exact in fp32 (8-bit x 8-bit significands) and the
 // RMS scale factor r multiplies a whole row, so it only adds a relative error.
-// The rotation of (x*gamma) uses cos/sin computed in fp64 and carried as float
-// pairs, with error-free products, which removes the absolute error a plain fp32
-// rotation has when its two terms cancel.  The result is therefore within a few
-// fp32 ulps (relative) of the exact value, i.e. within one bf16 ulp of its
-// correctly rounded bf16.  The kernel is HBM-bound: two reads and two writes of
-// n_tokens * n_heads * d bf16 values.
+// The rotation of a = x*gamma is the complex product a*c + (-a1, a0)*s with
+// cos and sin from fp64 carried as float pairs (hi + lo): the sine term's hi
+// product is split into its rounded value and exact error (fma), so the one
+// rounded sum a*c_hi + q is within 2^-24 of the result even where the two terms
+// cancel, and the small terms carry the rest.  The result is therefore within a
+// few fp32 ulps (relative) of the exact value, i.e. within one bf16 ulp of its
+// correctly rounded bf16.  Pairs of elements go through packed fp32 arithmetic
+// (two values per instruction), which halves the instructions the rotation and
+// the norm issue; three 256-thread blocks stay resident per SM.  The kernel is
+// HBM-bound: two reads and two writes of n_tokens * n_heads * d bf16 values.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -73,7 +77,7 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float (&y)[8]) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) prologue_kernel(const __grid_constant__ PrologueParams p) {
+__global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant__ PrologueParams p) {
   constexpr int kRowLanes = D / 8;             // lanes per row (16 B each)
   constexpr int kRowsPerPass = 32 / kRowLanes;  // rows per warp pass (Q/K interleaved)
   constexpr int kHeadsPerPass = kRowsPerPass / 2;
@@ -162,35 +166,48 @@ __global__ void __launch_bounds__(256) prologue_kernel(const __grid_constant__ P
       bf16x8_to_f32(raw[u], x);
       float r = 1.0f;
       if (any_norm) {  // warp-uniform: every lane joins the shuffles
-        float ss = 0.0f;
+        float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+        for (int i = 0; i < 4; ++i) {
+          const float2 xi = make_float2(x[2 * i], x[2 * i + 1]);
+          ss2 = __ffma2_rn(xi, xi, ss2);
+        }
+        float ss = ss2.x + ss2.y;
 #pragma unroll
         for (int off = kRowLanes / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         if (do_norm) {
           r = rsqrtf(fmaf(ss, inv_d, p.eps));
 #pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] *= g[i];  // exact
+          for (int i = 0; i < 4; ++i) {  // exact
+            const float2 xg = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), make_float2(g[2 * i], g[2 * i + 1]));
+            x[2 * i] = xg.x;
+            x[2 * i + 1] = xg.y;
+          }
         }
       }
       float y[8];
       if (do_rope) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          // (a0, a1) = x*gamma is exact in fp32.  Each product a*c_hi is split into
-          // its rounded value and exact error (fma), so the difference of the two
-          // large products is exact when they nearly cancel (Sterbenz) and the small
-          // terms carry the rest: the rotated value has a relative error of a few
-          // fp32 ulps even when its two terms cancel.
-          const float a0 = x[2 * k], a1 = x[2 * k + 1];
-          const float p0 = a0 * ch[k], e0 = fmaf(a0, ch[k], -p0);
-          const float q0 = a1 * sh[k], f0 = fmaf(a1, sh[k], -q0);
-          const float t0 = (p0 - q0) + (fmaf(a0, cl[k], e0) - fmaf(a1, sl[k], f0));
-          const float p1 = a0 * sh[k], e1 = fmaf(a0, sh[k], -p1);
-          const float q1 = a1 * ch[k], f1 = fmaf(a1, ch[k], -q1);
-          const float t1 = (p1 + q1) + (fmaf(a0, sl[k], e1) + fmaf(a1, cl[k], f1));
-          y[2 * k] = t0 * r;
-          y[2 * k + 1] = t1 * r;
+          // The pair a = (a0, a1) = x*gamma is exact in fp32.  As a complex product,
+          // y = a*c + ra*s with ra = (-a1, a0) and c, s each an unevaluated float pair
+          // (hi + lo).  The sine term's hi product is split into its rounded value q
+          // and exact error e (fma); m = a*c_hi + q then rounds once to within 2^-24
+          // of the result even where the two terms cancel, and the small terms
+          // (e, a*c_lo, ra*s_lo) carry the rest.  Each line works on both elements of
+          // the pair at once (packed fp32 pairs).
+          const float2 a = make_float2(x[2 * k], x[2 * k + 1]);
+          const float2 ra = make_float2(-x[2 * k + 1], x[2 * k]);
+          const float2 shi = make_float2(sh[k], sh[k]), slo = make_float2(sl[k], sl[k]);
+          const float2 chi = make_float2(ch[k], ch[k]), clo = make_float2(cl[k], cl[k]);
+          const float2 q = __fmul2_rn(ra, shi);
+          const float2 e = __ffma2_rn(ra, shi, make_float2(-q.x, -q.y));
+          const float2 m = __ffma2_rn(a, chi, q);
+          float2 lo = __ffma2_rn(a, clo, e);
+          lo = __ffma2_rn(ra, slo, lo);
+          const float2 yy = __fmul2_rn(__fadd2_rn(m, lo), make_float2(r, r));
+          y[2 * k] = yy.x;
+          y[2 * k + 1] = yy.y;
         }
       } else {
 #pragma unroll

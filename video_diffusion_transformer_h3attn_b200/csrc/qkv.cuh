@@ -25,10 +25,13 @@
 //     quarter) and 128 of the tile's 256 features; each thread one token row,
 //     32 accumulator columns at a time (a first pass over a Q/K head forms the
 //     sum of squares); results go through a per-warp 2 KB shared-memory block
-//     so that four lanes write each row's 64 bytes together.  Q/K heads: RMS in fp32, x * (1/rms) * gamma, then RoPE
-//     with the angle formed and reduced to [-pi, pi] in fp64 and cos/sin from
-//     the fp32 intrinsic (the projection's fp32 accumulation error dominates
-//     here, unlike in the standalone prologue whose input is exact); V: bias and
+//     (32 tokens x 32 features in the 64-byte swizzle), which the CTA-pair kernel
+//     writes out with one bulk tensor store per block and the single-CTA kernel
+//     with row-contiguous 16-byte stores (four lanes per row).  Q/K heads: RMS in fp32, x * (1/rms) * gamma, then RoPE
+//     with the angle formed and reduced to [-pi, pi] in fp32 with error-free
+//     products (frequency and 2 pi carried as float pairs) and cos/sin from the
+//     fp32 intrinsic (the projection's fp32 accumulation error dominates here,
+//     unlike in the standalone prologue whose input is exact); V: bias and
 //     rounding only.
 // Tiles are numbered feature-tile fastest, so the CTAs running at once share a
 // few X row blocks and W stays resident in L2 (3*H*d x dim_in bf16 = 57 MB at
@@ -113,10 +116,12 @@ struct QkvPairTraits {
   static constexpr int kBarriers = 2 * kStages + 5;
   static constexpr int kBarrierBytes = (8 * kBarriers + 15) / 16 * 16;
   static constexpr int kStageOutBytes = QkvTraits::kStageOutBytes;
+  // layout: stages | output staging blocks (1024-byte aligned: the 64-byte swizzle
+  // of the bulk tensor stores is taken from address bits) | barriers | slot words
   static constexpr int kSmemBytes =
-      1024 + kStages * kStageBytes + kBarrierBytes + 16 + kGemmEpiWarps * kStageOutBytes;
+      1024 + kStages * kStageBytes + kGemmEpiWarps * kStageOutBytes + kBarrierBytes + 16;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert((kStages * kStageBytes + kBarrierBytes + 16) % 16 == 0, "staging blocks 16-byte aligned");
+  static_assert((kStages * kStageBytes) % 1024 == 0, "staging blocks 1024-byte aligned");
 };
 constexpr int kGemmPairBM = 2 * kGemmBM;  // tokens per pair tile
 
@@ -125,9 +130,10 @@ constexpr int kGemmPairBM = 2 * kGemmBM;  // tokens per pair tile
 // features (`half`), read from tensor memory at tacc.  Q/K: bias, RMS norm, gamma,
 // RoPE; V: bias; all rounded once to bf16 and stored through the warp's staging
 // block wstage.
-template <int D>
+template <int D, bool kBulkStore = false>
 __device__ __forceinline__ void qkv_epilogue_tile(const QkvParams& p, int64_t m_row0, int nt, int quarter,
-                                                  int half, int lane, uint32_t tacc, uint8_t* wstage) {
+                                                  int half, int lane, uint32_t tacc, uint8_t* wstage,
+                                                  const CUtensorMap* const* out_maps = nullptr) {
   const int hd = p.n_heads * D;
   const int row = quarter * 32 + lane;  // token row inside the tile
   const int f0 = nt * kGemmBN + half * 128;  // first feature of this warp's 128
@@ -244,12 +250,28 @@ __device__ __forceinline__ void qkv_epilogue_tile(const QkvParams& p, int64_t m_
         // stage this thread's 32 columns (four 16-byte pieces of its row) in the
         // warp's block, pieces swizzled by row so that the writes and the
         // row-wise reads below are free of bank conflicts
+        if (kBulkStore) {  // the block's previous bulk store must have read it
+          if (lane == 0) ptx::bulk_wait_read_all();
+          __syncwarp();
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int sw = q ^ ((lane >> 1) & 3);
           *reinterpret_cast<uint4*>(wstage + lane * 64 + sw * 16) =
               make_uint4(ptx::pack_bf16x2(v[8 * q], v[8 * q + 1]), ptx::pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                          ptx::pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), ptx::pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        }
+        if (kBulkStore) {
+          // one bulk tensor store of the 32 x 32 block (the swizzle above is the
+          // tensor map's 64-byte swizzle); rows past the last token are clipped
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          const int64_t tok0 = m_row0 + quarter * 32;
+          if (lane == 0 && tok0 < p.n_tokens) {
+            ptx::tma_store_3d(out_maps[part], ptx::smem_u32(wstage), c, head, static_cast<int32_t>(tok0));
+            ptx::bulk_commit_group();
+          }
+          continue;
         }
         __syncwarp();
         // row-contiguous stores: lanes 4r..4r+3 write the 64 bytes of one row
@@ -433,21 +455,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     qkv_fused_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                          const __grid_constant__ QkvParams p) {
+                          const __grid_constant__ CUtensorMap tm_oq, const __grid_constant__ CUtensorMap tm_ok,
+                          const __grid_constant__ CUtensorMap tm_ov, const __grid_constant__ QkvParams p) {
   using T = QkvPairTraits;
   constexpr int kS = T::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* const base_ptr = smem_raw + (base - raw_addr);
-  const uint32_t bars = base + kS * T::kStageBytes;
+  const uint32_t bars = base + kS * T::kStageBytes + kGemmEpiWarps * T::kStageOutBytes;
   auto bar_full = [&](int s) { return bars + 8u * s; };
   auto bar_empty = [&](int s) { return bars + 8u * (kS + s); };
   auto bar_acc_full = [&](int b) { return bars + 8u * (2 * kS + b); };
   auto bar_acc_empty = [&](int b) { return bars + 8u * (2 * kS + 2 + b); };
   const uint32_t bar_drain = bars + 8u * (2 * kS + 4);  // MMA lane's exit after a failure
-  volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(base_ptr + kS * T::kStageBytes + T::kBarrierBytes);
-  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes + T::kBarrierBytes + 16;
+  uint8_t* const stage_out = base_ptr + kS * T::kStageBytes;
+  volatile uint32_t* const slot = reinterpret_cast<volatile uint32_t*>(
+      base_ptr + kS * T::kStageBytes + kGemmEpiWarps * T::kStageOutBytes + T::kBarrierBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -581,8 +605,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       ptx::tc_fence_after();
       const int m = tile / p.n_tiles, nt = tile % p.n_tiles;
       const uint32_t tacc = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kGemmBN + half * 128;
-      qkv_epilogue_tile<D>(p, static_cast<int64_t>(m) * kGemmPairBM + static_cast<int64_t>(rank) * kGemmBM, nt,
-                           quarter, half, lane, tacc, wstage);
+      const CUtensorMap* const maps[3] = {&tm_oq, &tm_ok, &tm_ov};
+      qkv_epilogue_tile<D, true>(p, static_cast<int64_t>(m) * kGemmPairBM + static_cast<int64_t>(rank) * kGemmBM,
+                                 nt, quarter, half, lane, tacc, wstage, maps);
       // the accumulator is read: rank 0's tensor core may reuse it
       ptx::tc_fence_before();
       __syncwarp();
@@ -590,6 +615,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  if (warp >= kGemmEpiWarp0 && lane == 0) ptx::bulk_wait_all();  // this warp's output stores are done
   __syncwarp();
   ptx::tc_fence_before();
   ptx::cluster_sync();  // no CTA leaves while its peer may still signal or read it
