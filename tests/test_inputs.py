@@ -1,5 +1,6 @@
 """The seeded input generator: determinism, shapes and layout of the workloads."""
 import numpy as np
+import pytest
 
 from video_diffusion_transformer_h3attn_b200 import inputs
 
@@ -92,3 +93,19 @@ def test_bench_sparse_flops_match_a_mask_count():
             for t in idx[off[c]:off[c + 1]]:
                 mask[h, 256 * qp:256 * (qp + 1), 128 * int(t):128 * (int(t) + 1)] = True
     assert flops == 4.0 * d * int(mask.sum())
+
+
+@pytest.mark.parametrize("lens", [[129024], [4096, 9000, 17001, 31234], [1, 130, 0, 255, 4, 513, 128], [300]])
+def test_sample_rows_every_tile_visits_every_query_tile(lens):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    rows = inputs.sample_rows_every_tile(cu, 64, seed=3)
+    assert np.all(np.diff(rows) > 0) and rows[0] >= 0 and rows[-1] < cu[-1]
+    for s in range(len(lens)):
+        a, b = int(cu[s]), int(cu[s + 1])
+        mine = rows[(rows >= a) & (rows < b)]
+        for t0 in range(a, b, 128):
+            assert np.any((mine >= t0) & (mine < min(t0 + 128, b))), "tile at %d of sequence %d not sampled" % (t0, s)
+        if b > a:
+            assert a in mine and b - 1 in mine
+    assert len(rows) >= min(64, int(cu[-1]))
+    assert np.array_equal(rows, inputs.sample_rows_every_tile(cu, 64, seed=3))
