@@ -672,6 +672,10 @@ def run_table(args):
         t_att = time.perf_counter() - t0
         got = (gpu_o if rows is None else gpu_o[rows]).astype(np.uint32) << 16
         err = np.abs(got.view(np.float32).astype(np.float64) - ro)
+        # the error beyond half a bf16 ulp of the exact value (what storing even the
+        # correctly rounded result in bf16 costs)
+        _, ex = np.frexp(np.maximum(np.abs(ro), 2.0 ** -126))
+        excess = np.maximum(err - np.ldexp(1.0, ex - 9), 0.0)
         frac = 1.0 if rows is None else len(rows) / w.total
         oracle_s = t_pro + t_att / frac
         tf = w.attention_flops() / (ms * 1e-3) / 1e12
@@ -687,6 +691,7 @@ def run_table(args):
             "prologue_gbs": prologue_bytes(w) / (pro_ms * 1e-3) / 1e9 if w.has_prologue else None,
             "prologue_max_ulp": max_ulp,
             "max_abs": float(err.max()), "mean_abs": float(err.mean()),
+            "max_abs_beyond_half_ulp": float(excess.max()),
             "compared": "every output" if rows is None else
                         "%d query rows x %d heads visiting every query tile" % (len(rows), w.n_heads),
             "oracle_s": oracle_s,
