@@ -132,3 +132,27 @@ def test_qkv_fused_matches_projection_then_prologue(h3):
     for a, b_ in ((q, q2), (k, k2), (v, proj[:, 2])):
         diff = (a.float() - b_.float()).abs()
         assert diff.max().item() < 0.08 and diff.mean().item() < 2e-3
+
+
+@pytest.mark.parametrize("n", [1, 33, 300])
+def test_qkv_fused_output_layouts_are_bitwise_identical(h3, n):
+    """The outputs leave through bulk tensor stores whose tensor maps are built from
+    the output strides: views of one fused [n, 3, H, d] buffer and head-outermost
+    views ([H, n, d] storage) give exactly the bits of separate contiguous outputs,
+    with a ragged last block of tokens (n not a multiple of 32) and a single token."""
+    import torch
+    H, d = 4, 128
+    x, w, b, gq, gk, pos, kind, sec = _case(n, 512, H, d, seed=70 + n)
+    xt, wt, bt = to_cuda_bf16(x), to_cuda_bf16(w), to_cuda_bf16(b)
+    g = (to_cuda_bf16(gq), to_cuda_bf16(gk))
+    pt, kt = torch.from_numpy(pos).cuda(), torch.from_numpy(kind).cuda()
+    kw = dict(bias=bt, gamma_q=g[0], gamma_k=g[1], pos=pt, kind=kt, sections=sec)
+    ref = h3.qkv_fused(xt, wt, H, **kw)
+    fused = torch.full((n, 3, H, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    got = h3.qkv_fused(xt, wt, H, q_out=fused[:, 0], k_out=fused[:, 1], v_out=fused[:, 2], **kw)
+    heads_out = [torch.full((H, n, d), 7.0, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    got2 = h3.qkv_fused(xt, wt, H, q_out=heads_out[0].permute(1, 0, 2), k_out=heads_out[1].permute(1, 0, 2),
+                        v_out=heads_out[2].permute(1, 0, 2), **kw)
+    h3.device_status()
+    for r, a, c in zip(ref, got, got2):
+        assert torch.equal(r, a) and torch.equal(r, c)
