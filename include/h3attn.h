@@ -31,7 +31,8 @@
  *   - Every device pointer and every stride must be a multiple of 16 bytes
  *     (strides: multiples of 8 elements); otherwise H3ATTN_ERR_MISALIGNED.
  *   - The caller owns every buffer.  The library allocates and frees no device
- *     memory; it holds one small static device word for error reporting.
+ *     memory; it holds two small static device words for error reporting (the
+ *     error word and the copy h3attn_device_status reads it through).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
  *     stream) of the current device and runs asynchronously: no call
  *     synchronises the device.  All argument checks happen on the host before
