@@ -65,7 +65,8 @@ def ulysses_attention(q, k, v, sizes: Sequence[int], group=None, *, gamma_q=None
                       eps: float = 1e-6, pos=None, kind=None, sections=(32, 48, 48),
                       theta: float = 10000.0, cu_seqlens=None, max_seqlen: Optional[int] = None,
                       softmax_scale: Optional[float] = None,
-                      prologue_fn: Optional[Callable] = None, attention_fn: Optional[Callable] = None):
+                      prologue_fn: Optional[Callable] = None, attention_fn: Optional[Callable] = None,
+                      exchange_fn: Optional[Callable] = None):
     """Sequence-parallel prologue + attention over P ranks of `group`.
 
     q, k, v: this rank's token shard [n_r, H, d] (bf16; q and k with equal
@@ -77,7 +78,10 @@ def ulysses_attention(q, k, v, sizes: Sequence[int], group=None, *, gamma_q=None
 
     prologue_fn / attention_fn replace the CUDA kernels (tests run the exchange
     on CPU ranks with reference implementations); by default the library's
-    kernels run.
+    kernels run.  exchange_fn(dst, src, out_splits, in_splits, group) replaces
+    torch.distributed.all_to_all_single (flat tensors, split sizes in elements),
+    e.g. a transport that stages device tensors through host memory for a
+    process group whose backend only moves host tensors.
     """
     import torch
     import torch.distributed as dist
@@ -96,6 +100,7 @@ def ulysses_attention(q, k, v, sizes: Sequence[int], group=None, *, gamma_q=None
     N = sum(sizes)
     prologue_fn = prologue_fn or _default_prologue
     attention_fn = attention_fn or _default_attention
+    exchange_fn = exchange_fn or dist.all_to_all_single
     dev, dt = q.device, q.dtype
 
     # 1. prologue fused with the pack: send blocks [P][n_r][Hp][d]
@@ -119,15 +124,14 @@ def ulysses_attention(q, k, v, sizes: Sequence[int], group=None, *, gamma_q=None
     out_splits = [s * Hp * d for s in sizes]
     in_splits = [n_r * Hp * d] * world
     for src, dst in zip((send_q, send_k, send_v), recv):
-        dist.all_to_all_single(dst.view(-1), src.view(-1), out_splits, in_splits, group=group)
+        exchange_fn(dst.view(-1), src.view(-1), out_splits, in_splits, group=group)
 
     # 3. attention over the whole sequence for this rank's heads
     o_heads = attention_fn(recv[0], recv[1], recv[2], cu_seqlens, max_seqlen, softmax_scale)
 
     # 4. head shards -> token shards, then unpack to [n_r][H][d]
     back = torch.empty((world, n_r, Hp, d), dtype=dt, device=dev)
-    dist.all_to_all_single(back.view(-1), o_heads.contiguous().view(-1), in_splits, out_splits,
-                           group=group)
+    exchange_fn(back.view(-1), o_heads.contiguous().view(-1), in_splits, out_splits, group=group)
     o = torch.empty((n_r, H, d), dtype=dt, device=dev)
     for p in range(world):
         o[:, p * Hp:(p + 1) * Hp].copy_(back[p])
