@@ -64,6 +64,17 @@ typedef enum {
 /* Library version as 10000*major + 100*minor + patch. */
 int h3attn_version(void);
 
+/*
+ * Build flags of the loaded library: H3ATTN_BUILD_DEBUG_BOUNDS is set in the
+ * debug build (compiled with H3ATTN_DEBUG_BOUNDS), where every kernel checks
+ * each global store's indices against its own launch's extents and, instead of
+ * storing out of place, records the failure for h3attn_device_status (which
+ * then returns H3ATTN_ERR_INVALID_ARG).  Release builds compile those checks
+ * away.  The checks stand in for a memory checker where none can run.
+ */
+#define H3ATTN_BUILD_DEBUG_BOUNDS 1
+int h3attn_build_flags(void);
+
 /* Static text for a status code (never NULL). */
 const char* h3attn_status_string(int status);
 
@@ -74,7 +85,8 @@ const char* h3attn_last_error(void);
  * Reads the device error word of the current device once the work already on
  * `stream` has finished, then synchronises `stream`: H3ATTN_OK;
  * H3ATTN_ERR_INVALID_ARG if a ragged launch's cu_seqlens or a block-sparse key
- * list broke its rules (h3attn_fwd_varlen, h3attn_fwd_block_sparse);
+ * list broke its rules (h3attn_fwd_varlen, h3attn_fwd_block_sparse), or, in a
+ * debug build, a bounds check fired;
  * H3ATTN_ERR_DEVICE_TIMEOUT if any kernel of this library gave up on a bounded
  * wait since the word was last cleared; H3ATTN_ERR_CUDA if the stream reports
  * an error.  The word is read and (clear != 0) zeroed by one atomic exchange

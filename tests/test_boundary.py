@@ -250,3 +250,15 @@ def test_binding_normalises_strides_of_size_one_dimensions():
     assert list(_strides2(t)) == [128, 8]
     t = torch.empty(2, 3, 4, 128)
     assert list(_strides3(t)) == [3 * 4 * 128, 4 * 128, 128]
+
+
+def test_debug_bounds_build_exports_the_same_calls():
+    """The bounds-checking debug build (H3ATTN_DEBUG_BOUNDS) exports every declared
+    call and says so in its build flags; the release build does not."""
+    import ctypes
+    _build.build(debug_bounds=True)
+    dbg = ctypes.CDLL(_build.DEBUG_LIBRARY)
+    for n in h3.declared_symbols():
+        assert hasattr(dbg, n), "debug library does not export %s" % n
+    assert dbg.h3attn_build_flags() == 1
+    assert h3.library().h3attn_build_flags() == 0

@@ -20,7 +20,8 @@ from typing import Optional, Sequence, Tuple
 from . import _build
 
 __all__ = ["prologue", "attention", "attention_varlen", "attention_kv", "attention_block_sparse", "merge",
-           "qkv_fused", "device_status", "selftest_wait_timeout", "library", "H3AttnError", "KIND_NONE", "KIND_3D", "KIND_1D",
+           "qkv_fused", "device_status", "selftest_wait_timeout", "library", "use_library", "build_flags",
+           "H3AttnError", "KIND_NONE", "KIND_3D", "KIND_1D",
            "declared_symbols"]
 
 KIND_NONE, KIND_3D, KIND_1D = 0, 1, 2
@@ -45,6 +46,19 @@ _I64_3 = ctypes.c_int64 * 3
 _I64_2 = ctypes.c_int64 * 2
 
 
+def use_library(path: Optional[str] = None) -> None:
+    """Load the library from `path` for the calls that follow (None: the release
+    build; _build.DEBUG_LIBRARY: the bounds-checking debug build)."""
+    global _lib, LIBRARY_PATH
+    LIBRARY_PATH = path or _build.LIBRARY
+    _lib = None
+
+
+def build_flags() -> int:
+    """h3attn_build_flags() of the loaded library (bit 1: bounds-checking debug build)."""
+    return int(library().h3attn_build_flags())
+
+
 def library() -> ctypes.CDLL:
     """The loaded libh3attn.so (raises if it has not been built)."""
     global _lib
@@ -54,6 +68,7 @@ def library() -> ctypes.CDLL:
                                "python -m video_diffusion_transformer_h3attn_b200._build" % LIBRARY_PATH)
         lib = ctypes.CDLL(LIBRARY_PATH)
         lib.h3attn_version.restype = ctypes.c_int
+        lib.h3attn_build_flags.restype = ctypes.c_int
         lib.h3attn_status_string.restype = ctypes.c_char_p
         lib.h3attn_status_string.argtypes = [ctypes.c_int]
         lib.h3attn_last_error.restype = ctypes.c_char_p

@@ -15,6 +15,9 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG_DIR, "libh3attn.so")
+# the same sources with H3ATTN_DEBUG_BOUNDS: every kernel checks its store indices
+# against its own launch's extents and reports instead of storing out of place
+DEBUG_LIBRARY = os.path.join(PKG_DIR, "libh3attn_debug.so")
 MAIN_SOURCE = os.path.join(CSRC, "h3attn_api.cu")
 
 NVCC_FLAGS = [
@@ -42,12 +45,17 @@ def needs_build(output: str = LIBRARY) -> bool:
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, output: str = LIBRARY, verbose: bool = False) -> str:
-    """Compile libh3attn.so in place (skipped when it is newer than every source)."""
+def build(force: bool = False, output: str = LIBRARY, verbose: bool = False, debug_bounds: bool = False) -> str:
+    """Compile libh3attn.so (or, with debug_bounds, libh3attn_debug.so) in place;
+    skipped when the library is newer than every source."""
+    if debug_bounds and output == LIBRARY:
+        output = DEBUG_LIBRARY
     if not force and not needs_build(output):
         return output
     tmp = output + ".tmp%d" % os.getpid()
     cmd = [_nvcc(), *NVCC_FLAGS, "-I" + INCLUDE, "-o", tmp, MAIN_SOURCE]
+    if debug_bounds:
+        cmd.insert(1, "-DH3ATTN_DEBUG_BOUNDS")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

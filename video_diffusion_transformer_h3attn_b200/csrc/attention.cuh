@@ -236,7 +236,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // no keys (a block of a split key set may be empty): the empty sum, O = 0 and
     // LSE = -inf, for the CTA's rows; nothing else runs
     const int64_t row = q_row0 + threadIdx.x;
-    if (threadIdx.x < kQTiles * kBM && row < seq_len) {
+    if (threadIdx.x < kQTiles * kBM && row < seq_len &&
+        store_in_bounds(seq_base + row < (kVarlen ? p.total : p.seqlen) && head < p.n_heads &&
+                        batch < static_cast<int>(gridDim.z))) {
       uint4* orow = reinterpret_cast<uint4*>(p.o + static_cast<int64_t>(batch) * p.o_batch +
                                              (seq_base + row) * p.o_tok + static_cast<int64_t>(head) * p.o_head);
 #pragma unroll
@@ -620,7 +622,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
       ptx::tc_fence_after();
       const int64_t row0 = q_row0 + t * kBM + r0, row1 = q_row0 + t * kBM + r1;  // within the sequence
-      const bool v0 = row0 < seq_len, v1 = row1 < seq_len;
+      const int64_t tok_extent = kVarlen ? p.total : p.seqlen;  // token rows of O and of each LSE row
+      const bool in_launch = head < p.n_heads && batch < static_cast<int>(gridDim.z);
+      const bool v0 = row0 < seq_len && store_in_bounds(in_launch && seq_base + row0 < tok_extent);
+      const bool v1 = row1 < seq_len && store_in_bounds(in_launch && seq_base + row1 < tok_extent);
       const float inv0 = 1.0f / l0, inv1 = 1.0f / l1;
       uint16_t* const obase = p.o + static_cast<int64_t>(batch) * p.o_batch + static_cast<int64_t>(head) * p.o_head;
       uint32_t* const o0 = reinterpret_cast<uint32_t*>(obase + (seq_base + row0) * p.o_tok) + cq;

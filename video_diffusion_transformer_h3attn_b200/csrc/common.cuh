@@ -13,6 +13,7 @@ enum : uint32_t {
   kErrTimeout = 1u,       // a bounded wait gave up
   kErrBadBlockList = 2u,  // a block-sparse key list was not strictly ascending in range
   kErrBadSeqlens = 4u,    // a ragged launch's cu_seqlens broke its rules (the launch wrote nothing)
+  kErrBounds = 8u,        // debug builds: a store index outside the launch's own extents (skipped)
 };
 
 // Device error word: [0] = sticky error bits, [1] = id of the last launch that
@@ -44,6 +45,23 @@ __device__ __forceinline__ bool launch_failed(const LaunchCtl& ctl) {
 
 // An error that leaves the rest of the launch running (no launch id recorded).
 __device__ __forceinline__ void report_error(uint32_t bits) { atomicOr(&g_error_word[0], bits); }
+
+// Debug builds (compiled with H3ATTN_DEBUG_BOUNDS) check every global store's
+// indices against the extents of the launch that makes it: an index outside them
+// records kErrBounds and the store is skipped (no trap, nothing written out of
+// place).  Release builds compile the check away.
+#ifdef H3ATTN_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool store_in_bounds(bool in_bounds) {
+  if (kDebugBounds && !in_bounds) {
+    atomicOr(&g_error_word[0], kErrBounds);
+    return false;
+  }
+  return true;
+}
 
 __device__ __forceinline__ void report_failure(const LaunchCtl& ctl, uint32_t bits) {
   atomicOr(&g_error_word[0], bits);

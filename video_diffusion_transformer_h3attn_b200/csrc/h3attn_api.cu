@@ -272,6 +272,8 @@ extern "C" {
 
 int h3attn_version(void) { return kVersion; }
 
+int h3attn_build_flags(void) { return h3::kDebugBounds ? H3ATTN_BUILD_DEBUG_BOUNDS : 0; }
+
 const char* h3attn_status_string(int status) {
   switch (status) {
     case H3ATTN_OK: return "ok";
@@ -302,6 +304,10 @@ int h3attn_device_status(void* stream, int clear) {
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if (word[0] & h3::kErrBounds)
+    return fail(H3ATTN_ERR_INVALID_ARG,
+                "a debug bounds check fired: a kernel computed a store index outside its launch's extents "
+                "(the store was skipped)");
   if (word[0] & h3::kErrBadSeqlens)
     return fail(H3ATTN_ERR_INVALID_ARG,
                 "cu_seqlens broke its rules (cu[0] = 0, non-decreasing, lengths <= max_seqlen, "

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
         wa = ea / sum;
         wb = eb / sum;
       }
-      p.lse[lrow + n] = L;
+      if (store_in_bounds(head < p.n_heads && batch < static_cast<int64_t>(gridDim.z))) p.lse[lrow + n] = L;
     }
     s_wa[threadIdx.x] = wa;
     s_wb[threadIdx.x] = wb;
@@ -88,8 +88,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const __grid_const
       const float b_lo = __uint_as_float(b[i] << 16), b_hi = __uint_as_float(b[i] & 0xFFFF0000u);
       out[i] = ptx::pack_bf16x2(fmaf(wa, a_lo, wb * b_lo), fmaf(wa, a_hi, wb * b_hi));
     }
-    *reinterpret_cast<uint4*>(p.o + batch * p.o_batch + n * p.o_tok + head * p.o_head + chunk * 8) =
-        make_uint4(out[0], out[1], out[2], out[3]);
+    if (store_in_bounds(n < p.seqlen && head < p.n_heads && batch < static_cast<int64_t>(gridDim.z) &&
+                        chunk * 8 + 8 <= D))
+      *reinterpret_cast<uint4*>(p.o + batch * p.o_batch + n * p.o_tok + head * p.o_head + chunk * 8) =
+          make_uint4(out[0], out[1], out[2], out[3]);
   }
 }
 

@@ -213,8 +213,8 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant_
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = x[i] * r;
       }
-      if (live[u]) {
-        const int h = (pass0 + u) * kHeadsPerPass + head_in_pass;
+      const int h = (pass0 + u) * kHeadsPerPass + head_in_pass;
+      if (live[u] && store_in_bounds(token < p.n_tokens && h < n_heads && chunk * 8 + 8 <= D)) {
         *reinterpret_cast<uint4*>(dst + token * p.out_tok + h * p.out_head + chunk * 8) =
             f32x8_to_bf16(y);
       }

@@ -267,7 +267,7 @@ __device__ __forceinline__ void qkv_epilogue_tile(const QkvParams& p, int64_t m_
           ptx::fence_proxy_async_smem();
           __syncwarp();
           const int64_t tok0 = m_row0 + quarter * 32;
-          if (lane == 0 && tok0 < p.n_tokens) {
+          if (lane == 0 && tok0 < p.n_tokens && store_in_bounds(head < p.n_heads && c + 32 <= D)) {
             ptx::tma_store_3d(out_maps[part], ptx::smem_u32(wstage), c, head, static_cast<int32_t>(tok0));
             ptx::bulk_commit_group();
           }
@@ -281,7 +281,7 @@ __device__ __forceinline__ void qkv_epilogue_tile(const QkvParams& p, int64_t m_
           const int64_t tok = m_row0 + quarter * 32 + srow;
           const uint4 val =
               *reinterpret_cast<const uint4*>(wstage + srow * 64 + (piece ^ ((srow >> 1) & 3)) * 16);
-          if (tok < p.n_tokens) {
+          if (tok < p.n_tokens && store_in_bounds(head < p.n_heads && c + 32 <= D && part < 3)) {
             uint16_t* const drow = p.out[part] + tok * p.out_tok[part] +
                                    static_cast<int64_t>(head) * p.out_head[part] + c;
             *reinterpret_cast<uint4*>(drow + piece * 8) = val;
