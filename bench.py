@@ -692,6 +692,8 @@ def run_table(args):
             "prologue_max_ulp": max_ulp,
             "max_abs": float(err.max()), "mean_abs": float(err.mean()),
             "max_abs_beyond_half_ulp": float(excess.max()),
+            "n_over_1e-2": int(np.sum(err > 1e-2)), "n_over_1e-2_beyond_half_ulp": int(np.sum(excess > 1e-2)),
+            "n_compared": int(err.size),
             "compared": "every output" if rows is None else
                         "%d query rows x %d heads visiting every query tile" % (len(rows), w.n_heads),
             "oracle_s": oracle_s,
