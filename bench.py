@@ -665,17 +665,34 @@ def run_table(args):
                 return np.where(x & 0x8000, -(x & 0x7FFF), x & 0x7FFF)
             max_ulp = int(max(np.abs(ordered(gpu_qp) - ordered(q16)).max(),
                               np.abs(ordered(gpu_kp) - ordered(k16)).max()))
+        # the attention kernel alone on the oracle's own Q', K' (the same inputs on both sides)
+        dq = {"q": _bf16(q16).to(dev), "k": _bf16(k16).to(dev), "v": _bf16(w.v).to(dev)}
+        if len(w.seqlens) > 1:
+            o_same = h3.attention_varlen(dq["q"], dq["k"], dq["v"], torch.from_numpy(
+                np.ascontiguousarray(w.cu_seqlens, dtype=np.int32)).to(dev), w.max_seqlen)
+        else:
+            o_same = h3.attention(dq["q"], dq["k"], dq["v"])
+        h3.device_status()
+        gpu_o_same = o_same.view(torch.int16).cpu().numpy().view(np.uint16)
+        del dq, o_same
+        torch.cuda.empty_cache()
         n_rows = TABLE_SAMPLED_ROWS.get(name)
         rows = None if n_rows is None else inputs.sample_rows_every_tile(w.cu_seqlens, n_rows, seed=w.seed + 1000)
         t0 = time.perf_counter()
         ro, _ = orc.attention(q16, k16, w.v, w.cu_seqlens, rows=rows)
         t_att = time.perf_counter() - t0
-        got = (gpu_o if rows is None else gpu_o[rows]).astype(np.uint32) << 16
-        err = np.abs(got.view(np.float32).astype(np.float64) - ro)
         # the error beyond half a bf16 ulp of the exact value (what storing even the
         # correctly rounded result in bf16 costs)
         _, ex = np.frexp(np.maximum(np.abs(ro), 2.0 ** -126))
-        excess = np.maximum(err - np.ldexp(1.0, ex - 9), 0.0)
+        half_ulp = np.ldexp(1.0, ex - 9)
+
+        def errors(bits):
+            got = (bits if rows is None else bits[rows]).astype(np.uint32) << 16
+            e = np.abs(got.view(np.float32).astype(np.float64) - ro)
+            return e, np.maximum(e - half_ulp, 0.0)
+
+        err, excess = errors(gpu_o)
+        err_same, excess_same = errors(gpu_o_same)
         frac = 1.0 if rows is None else len(rows) / w.total
         oracle_s = t_pro + t_att / frac
         tf = w.attention_flops() / (ms * 1e-3) / 1e12
@@ -694,6 +711,13 @@ def run_table(args):
             "max_abs_beyond_half_ulp": float(excess.max()),
             "n_over_1e-2": int(np.sum(err > 1e-2)), "n_over_1e-2_beyond_half_ulp": int(np.sum(excess > 1e-2)),
             "n_compared": int(err.size),
+            "errors_above": "the step end to end: GPU prologue + attention against the oracle's prologue + attention",
+            "attention_same_inputs": {
+                "max_abs": float(err_same.max()), "mean_abs": float(err_same.mean()),
+                "max_abs_beyond_half_ulp": float(excess_same.max()),
+                "n_over_1e-2": int(np.sum(err_same > 1e-2)),
+                "n_over_1e-2_beyond_half_ulp": int(np.sum(excess_same > 1e-2)),
+                "note": "the attention kernel on the oracle's own Q', K' (identical inputs on both sides)"},
             "compared": "every output" if rows is None else
                         "%d query rows x %d heads visiting every query tile" % (len(rows), w.n_heads),
             "oracle_s": oracle_s,

@@ -23,7 +23,7 @@
 //     memory lanes and reads them with the 16x256b shape, so each query row's
 //     128 scores sit in four threads of one warp (32 each): row maxima and sums
 //     are two shuffles away, and two warps per scheduler work on each tile.  The
-//     running max m (log2 units) may lag the true max by < 8, so P <= 256 and O
+//     running max m (log2 units) may lag the true max by < 16, so P <= 2^16 and O
 //     is rescaled in tensor memory only when the max grows by more.  The first
 //     half of P is computed with m as it stands while the tile's maxima are
 //     formed, and redone only when m must grow, so the max is off the step's
@@ -58,7 +58,12 @@ constexpr int kMmaWarp = 17;
 constexpr int kAttnThreads = 640;
 // Registers: 640 threads launch at 96 per thread (five warps per scheduler x 96 <= 512);
 // a softmax thread holds 64 scores, so every role fits without a setmaxnreg split.
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+// log2 units: m is raised (and O rescaled) only when a row's maximum exceeds it by more
+// than this, so P <= 2^16: far inside bf16 and fp32 range (O and l stay below
+// n_keys * 2^16 * max|v|), and rows whose maximum creeps up in small steps (sharp
+// softmax rows) rarely take the slow path.  A row whose running max is exact has its
+// dominant weight exactly 1; with a lag that weight is rounded to bf16 like the rest.
+constexpr float kRescaleThreshold = 16.0f;
 constexpr int kSortMax = 256;              // ragged batches up to this many sequences run longest first
 
 template <int D>
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tO = tmem + lane_off + 256 + t * D;
     const float c = p.scale_log2;
     const float2 c2 = make_float2(c, c);
-    float m0 = -INFINITY, m1 = -INFINITY;  // running row maxima of s*c (log2), may lag by < 8
+    float m0 = -INFINITY, m1 = -INFINITY;  // running row maxima of s*c (log2), may lag by < 16
     float l0 = 0.0f, l1 = 0.0f;            // this thread's partial sums of bf16(2^(s*c - m))
     float lx0 = 0.0f, lx1 = 0.0f;          // the same in fp32 (log-sum-exp)
     bool ok = true;
