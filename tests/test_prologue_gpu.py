@@ -139,3 +139,22 @@ def test_prologue_many_heads(h3, orc, H, d):
     rq, rk = _ref(orc, w)
     check_prologue(gq, rq, "H%d q" % H)
     check_prologue(gk, rk, "H%d k" % H)
+
+
+@pytest.mark.parametrize("H,d", [(1, 128), (7, 128), (8, 128), (9, 128), (17, 128),
+                                 (1, 64), (15, 64), (16, 64), (17, 64), (33, 64)])
+def test_prologue_pass_counts(h3, orc, H, d):
+    # a warp streams its token's head passes (one head per pass at d = 128, two at
+    # d = 64) through a ring of eight: fewer passes than the ring, exactly the ring,
+    # one more, and several turns of it, with a half-live last pass at odd d = 64
+    # head counts; 45 tokens leave the last block's warps partly idle
+    n = 45
+    w = inputs.make_workload("passes%d_%d" % (H, d), [n], H, d, seed=300 + H + d, norm=True,
+                             sections=(32, 48, 48) if d == 128 else (16, 24, 24))
+    rng = np.random.default_rng(301 + H)
+    w.pos = np.stack([rng.integers(0, 40, n), rng.integers(0, 50, n), rng.integers(0, 5000, n)], 1).astype(np.int32)
+    w.kind = rng.integers(0, 3, n).astype(np.uint8)
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "H%d d%d q" % (H, d))
+    check_prologue(gk, rk, "H%d d%d k" % (H, d))

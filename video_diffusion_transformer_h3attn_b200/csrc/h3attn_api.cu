@@ -369,8 +369,8 @@ h3attn_status h3attn_prologue(const void* q_in, const void* k_in, void* q_out, v
   prm.n_heads = n_heads;
   prm.eps = static_cast<float>(eps);
 
-  constexpr int kThreads = 256;
-  constexpr int kTokensPerBlock = kThreads / 32;
+  constexpr int kThreads = h3::kPrologueThreads;
+  constexpr int kTokensPerBlock = kThreads / 32;  // one warp per token
   const int64_t blocks = (n_tokens + kTokensPerBlock - 1) / kTokensPerBlock;
   if (blocks > 0x7FFFFFFF) return fail(H3ATTN_ERR_UNSUPPORTED, "too many tokens");
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -10,8 +10,12 @@
 // (Q_h, K_h) for d = 128 or (Q_h, K_h, Q_h+1, K_h+1) for d = 64.  Loads and
 // stores are 128-bit and coalesced per row; the sum of squares is a shuffle
 // reduction inside each row's lane group; a lane owns whole rotation pairs, so
-// RoPE needs no data exchange.  The cos/sin of the token's pairs are computed
-// once per token in fp64 and reused by every head of Q and K.
+// the rotation itself needs no data exchange.  The cos/sin of the token's pairs
+// are computed once per token in fp64 (each pair by one of the lanes that share
+// it, then handed round by shuffles) and reused by every head of Q and K.  The
+// rows reach the warp through a per-warp ring in shared memory filled by 16-byte
+// cp.async copies several passes ahead, so many rows are in flight per warp
+// without holding registers for them.
 //
 // Precision: x*gamma is exact in fp32 (8-bit x 8-bit significands) and the
 // RMS scale factor r multiplies a whole row, so it only adds a relative error.
@@ -23,7 +27,8 @@
 // few fp32 ulps (relative) of the exact value, i.e. within one bf16 ulp of its
 // correctly rounded bf16.  Pairs of elements go through packed fp32 arithmetic
 // (two values per instruction), which halves the instructions the rotation and
-// the norm issue; three 256-thread blocks stay resident per SM.  The kernel is
+// the norm issue; four 256-thread blocks stay resident per SM (64 registers, 32 KB
+// of ring each).  The kernel is
 // HBM-bound: two reads and two writes of n_tokens * n_heads * d bf16 values.
 #pragma once
 
@@ -76,15 +81,32 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float (&y)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 16-byte asynchronous global -> shared copy (bypasses the register file and L1).
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_u32(dst_smem)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int kPrologueThreads = 256;
+constexpr int kPrologueDepth = 8;  // passes in flight per warp
+
 template <int D>
-__global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant__ PrologueParams p) {
-  constexpr int kRowLanes = D / 8;             // lanes per row (16 B each)
+__global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const __grid_constant__ PrologueParams p) {
+  constexpr int kRowLanes = D / 8;              // lanes per row (16 B each)
   constexpr int kRowsPerPass = 32 / kRowLanes;  // rows per warp pass (Q/K interleaved)
   constexpr int kHeadsPerPass = kRowsPerPass / 2;
-  constexpr int kUnroll = 4;
+  constexpr int kPairsPerLane = 4 / kRowsPerPass;  // sincos each lane evaluates (of its chunk's 4 pairs)
+  constexpr int kWarps = kPrologueThreads / 32;
+  // Each warp streams its token's rows through a ring of kPrologueDepth passes in shared
+  // memory (one 16-byte slot per lane and pass): a lane copies and later reads only its own
+  // slot, so its own cp.async groups order the ring and no barrier is needed.
+  __shared__ uint4 ring[kWarps][kPrologueDepth][32];
 
   const int lane = threadIdx.x & 31;
-  const int64_t token = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int warp = threadIdx.x >> 5;
+  const int64_t token = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
   if (token >= p.n_tokens) return;
 
   const int group = lane / kRowLanes;     // which row of the pass
@@ -92,9 +114,19 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant_
   const bool is_k = (group & 1) != 0;
   const int head_in_pass = group >> 1;
 
-  const uint16_t* src = is_k ? p.k_in : p.q_in;
-  uint16_t* dst = is_k ? p.k_out : p.q_out;
+  const uint16_t* src = (is_k ? p.k_in : p.q_in) + token * p.in_tok + chunk * 8;
+  uint16_t* dst = (is_k ? p.k_out : p.q_out) + token * p.out_tok + chunk * 8;
   const uint16_t* gamma = is_k ? p.gamma_k : p.gamma_q;
+  const int n_heads = p.n_heads;
+  const int n_pass = (n_heads + kHeadsPerPass - 1) / kHeadsPerPass;
+
+  // The first passes' rows are in flight while the token's angles are evaluated.
+#pragma unroll
+  for (int s = 0; s < kPrologueDepth; ++s) {
+    const int h = s * kHeadsPerPass + head_in_pass;
+    if (s < n_pass && h < n_heads) cp_async16(&ring[warp][s][lane], src + h * p.in_head);
+    cp_async_commit();
+  }
 
   // gamma of this lane's 8 elements (fp32, exact)
   float g[8];
@@ -104,7 +136,6 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant_
     bf16x8_to_f32(*reinterpret_cast<const uint4*>(gamma + chunk * 8), g);
   }
 
-  // cos/sin of this lane's 4 pairs for this token (fp64)
   int kind = 0;
   int32_t pt = 0, ph = 0, pw = 0;
   if (p.pos != nullptr) {
@@ -117,15 +148,17 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant_
       kind = 0;
     }
   }
-  const bool do_rope = kind != 0;
-  // cos and sin as unevaluated float pairs (hi + lo, |lo| <= ulp(hi)/2): the
-  // rotation below then runs in fp32 with error-free products, avoiding per-element
-  // fp32 <-> fp64 conversions (which share the slow conversion pipe).
+  const bool do_rope = kind != 0;  // warp-uniform (one token per warp)
+  // cos and sin of this lane's 4 rotation pairs as unevaluated float pairs (hi + lo,
+  // |lo| <= ulp(hi)/2), from fp64: the rotation below then runs in fp32 with error-free
+  // products.  The kRowsPerPass lanes that share a chunk need the same 4 pairs, so each
+  // evaluates kPairsPerLane of them and the four values per pair are exchanged by shuffles.
   float ch[4], cl[4], sh[4], sl[4];
   if (do_rope) {
+    float mch[kPairsPerLane], mcl[kPairsPerLane], msh[kPairsPerLane], msl[kPairsPerLane];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int pair = chunk * 4 + k;
+    for (int k = 0; k < kPairsPerLane; ++k) {
+      const int pair = chunk * 4 + group * kPairsPerLane + k;
       double angle;
       if (kind == 1) {
         const int ax = p.rope.axis_3d[pair];
@@ -136,89 +169,90 @@ __global__ void __launch_bounds__(256, 3) prologue_kernel(const __grid_constant_
       }
       double sd, cd;
       sincos(angle, &sd, &cd);
-      ch[k] = static_cast<float>(cd);
-      cl[k] = static_cast<float>(cd - static_cast<double>(ch[k]));
-      sh[k] = static_cast<float>(sd);
-      sl[k] = static_cast<float>(sd - static_cast<double>(sh[k]));
+      mch[k] = static_cast<float>(cd);
+      mcl[k] = static_cast<float>(cd - static_cast<double>(mch[k]));
+      msh[k] = static_cast<float>(sd);
+      msl[k] = static_cast<float>(sd - static_cast<double>(msh[k]));
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int from = (k / kPairsPerLane) * kRowLanes + chunk;  // the lane that evaluated pair chunk*4+k
+      ch[k] = __shfl_sync(0xffffffffu, mch[k % kPairsPerLane], from);
+      cl[k] = __shfl_sync(0xffffffffu, mcl[k % kPairsPerLane], from);
+      sh[k] = __shfl_sync(0xffffffffu, msh[k % kPairsPerLane], from);
+      sl[k] = __shfl_sync(0xffffffffu, msl[k % kPairsPerLane], from);
     }
   }
 
   const float inv_d = 1.0f / static_cast<float>(D);
-  const int n_heads = p.n_heads;
-  const int n_pass = (n_heads + kHeadsPerPass - 1) / kHeadsPerPass;
+  for (int pass = 0; pass < n_pass; ++pass) {
+    const int slot = pass % kPrologueDepth;
+    const int h = pass * kHeadsPerPass + head_in_pass;
+    const bool live = h < n_heads;
+    cp_async_wait<kPrologueDepth - 1>();  // this pass's group has landed
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (live) raw = ring[warp][slot][lane];
 
-  for (int pass0 = 0; pass0 < n_pass; pass0 += kUnroll) {
-    uint4 raw[kUnroll];
-    bool live[kUnroll];
+    float x[8];
+    bf16x8_to_f32(raw, x);
+    float r = 1.0f;
+    if (any_norm) {  // warp-uniform: every lane joins the shuffles
+      float2 ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int h = (pass0 + u) * kHeadsPerPass + head_in_pass;
-      live[u] = (pass0 + u) < n_pass && h < n_heads;
-      if (live[u]) {
-        raw[u] = *reinterpret_cast<const uint4*>(src + token * p.in_tok + h * p.in_head + chunk * 8);
-      } else {
-        raw[u] = make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) {
+        const float2 xi = make_float2(x[2 * i], x[2 * i + 1]);
+        ss2 = __ffma2_rn(xi, xi, ss2);
+      }
+      float ss = ss2.x + ss2.y;
+#pragma unroll
+      for (int off = kRowLanes / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (do_norm) {
+        r = rsqrtf(fmaf(ss, inv_d, p.eps));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // exact
+          const float2 xg = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), make_float2(g[2 * i], g[2 * i + 1]));
+          x[2 * i] = xg.x;
+          x[2 * i + 1] = xg.y;
+        }
       }
     }
+    float y[8];
+    if (do_rope) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      float x[8];
-      bf16x8_to_f32(raw[u], x);
-      float r = 1.0f;
-      if (any_norm) {  // warp-uniform: every lane joins the shuffles
-        float2 ss2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 xi = make_float2(x[2 * i], x[2 * i + 1]);
-          ss2 = __ffma2_rn(xi, xi, ss2);
-        }
-        float ss = ss2.x + ss2.y;
-#pragma unroll
-        for (int off = kRowLanes / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        if (do_norm) {
-          r = rsqrtf(fmaf(ss, inv_d, p.eps));
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {  // exact
-            const float2 xg = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), make_float2(g[2 * i], g[2 * i + 1]));
-            x[2 * i] = xg.x;
-            x[2 * i + 1] = xg.y;
-          }
-        }
+      for (int k = 0; k < 4; ++k) {
+        // The pair a = (a0, a1) = x*gamma is exact in fp32.  As a complex product,
+        // y = a*c + ra*s with ra = (-a1, a0) and c, s each an unevaluated float pair
+        // (hi + lo).  The sine term's hi product is split into its rounded value q
+        // and exact error e (fma); m = a*c_hi + q then rounds once to within 2^-24
+        // of the result even where the two terms cancel, and the small terms
+        // (e, a*c_lo, ra*s_lo) carry the rest.  Each line works on both elements of
+        // the pair at once (packed fp32 pairs).
+        const float2 a = make_float2(x[2 * k], x[2 * k + 1]);
+        const float2 ra = make_float2(-x[2 * k + 1], x[2 * k]);
+        const float2 shi = make_float2(sh[k], sh[k]), slo = make_float2(sl[k], sl[k]);
+        const float2 chi = make_float2(ch[k], ch[k]), clo = make_float2(cl[k], cl[k]);
+        const float2 q = __fmul2_rn(ra, shi);
+        const float2 e = __ffma2_rn(ra, shi, make_float2(-q.x, -q.y));
+        const float2 m = __ffma2_rn(a, chi, q);
+        float2 lo = __ffma2_rn(a, clo, e);
+        lo = __ffma2_rn(ra, slo, lo);
+        const float2 yy = __fmul2_rn(__fadd2_rn(m, lo), make_float2(r, r));
+        y[2 * k] = yy.x;
+        y[2 * k + 1] = yy.y;
       }
-      float y[8];
-      if (do_rope) {
+    } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          // The pair a = (a0, a1) = x*gamma is exact in fp32.  As a complex product,
-          // y = a*c + ra*s with ra = (-a1, a0) and c, s each an unevaluated float pair
-          // (hi + lo).  The sine term's hi product is split into its rounded value q
-          // and exact error e (fma); m = a*c_hi + q then rounds once to within 2^-24
-          // of the result even where the two terms cancel, and the small terms
-          // (e, a*c_lo, ra*s_lo) carry the rest.  Each line works on both elements of
-          // the pair at once (packed fp32 pairs).
-          const float2 a = make_float2(x[2 * k], x[2 * k + 1]);
-          const float2 ra = make_float2(-x[2 * k + 1], x[2 * k]);
-          const float2 shi = make_float2(sh[k], sh[k]), slo = make_float2(sl[k], sl[k]);
-          const float2 chi = make_float2(ch[k], ch[k]), clo = make_float2(cl[k], cl[k]);
-          const float2 q = __fmul2_rn(ra, shi);
-          const float2 e = __ffma2_rn(ra, shi, make_float2(-q.x, -q.y));
-          const float2 m = __ffma2_rn(a, chi, q);
-          float2 lo = __ffma2_rn(a, clo, e);
-          lo = __ffma2_rn(ra, slo, lo);
-          const float2 yy = __fmul2_rn(__fadd2_rn(m, lo), make_float2(r, r));
-          y[2 * k] = yy.x;
-          y[2 * k + 1] = yy.y;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = x[i] * r;
-      }
-      const int h = (pass0 + u) * kHeadsPerPass + head_in_pass;
-      if (live[u] && store_in_bounds(token < p.n_tokens && h < n_heads && chunk * 8 + 8 <= D)) {
-        *reinterpret_cast<uint4*>(dst + token * p.out_tok + h * p.out_head + chunk * 8) =
-            f32x8_to_bf16(y);
-      }
+      for (int i = 0; i < 8; ++i) y[i] = x[i] * r;
     }
+    if (live && store_in_bounds(token < p.n_tokens && h < n_heads && chunk * 8 + 8 <= D)) {
+      *reinterpret_cast<uint4*>(dst + h * p.out_head) = f32x8_to_bf16(y);
+    }
+    // Refill this slot (its value is consumed above) with the pass kPrologueDepth ahead; an
+    // empty group keeps the group count in step at the tail.
+    const int nxt = pass + kPrologueDepth;
+    const int hn = nxt * kHeadsPerPass + head_in_pass;
+    if (nxt < n_pass && hn < n_heads) cp_async16(&ring[warp][slot][lane], src + hn * p.in_head);
+    cp_async_commit();
   }
 }
 
