@@ -158,3 +158,18 @@ def test_prologue_pass_counts(h3, orc, H, d):
     rq, rk = _ref(orc, w)
     check_prologue(gq, rq, "H%d d%d q" % (H, d))
     check_prologue(gk, rk, "H%d d%d k" % (H, d))
+
+
+@pytest.mark.parametrize("sections", [(64, 64, 0), (0, 0, 128), (0, 128, 0), (32, 48, 48)])
+def test_prologue_video_rows_sections(h3, orc, sections):
+    # video rows of 16 tokens (tokens of a row share t and h); degenerate sections put
+    # every rotation pair on the t and h axes, or all on w, or all on h; 5 audio
+    # tokens end the clip
+    pos, kind = inputs.video_layout(3, 4, 16, n_audio=5)
+    n = len(pos)
+    w = inputs.make_workload("rows%d%d%d" % sections, [n], 6, 128, seed=400, norm=True, sections=sections,
+                             pos=pos, kind=kind)
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "sections %s q" % (sections,))
+    check_prologue(gk, rk, "sections %s k" % (sections,))

@@ -19,17 +19,18 @@
 //
 // Precision: x*gamma is exact in fp32 (8-bit x 8-bit significands) and the
 // RMS scale factor r multiplies a whole row, so it only adds a relative error.
-// The rotation of a = x*gamma is the complex product a*c + (-a1, a0)*s with
+// The rotation of (a0, a1) = x*gamma is y0 = a0*c - a1*s, y1 = a1*c + a0*s with
 // cos and sin from fp64 carried as float pairs (hi + lo): the sine term's hi
-// product is split into its rounded value and exact error (fma), so the one
-// rounded sum a*c_hi + q is within 2^-24 of the result even where the two terms
-// cancel, and the small terms carry the rest.  The result is therefore within a
+// product is split into its rounded value q and exact error (fma), so the one
+// rounded sum (cosine term's hi product) + q is within 2^-24 of the result even
+// where the two terms cancel, and the small terms carry the rest.  The result is therefore within a
 // few fp32 ulps (relative) of the exact value, i.e. within one bf16 ulp of its
-// correctly rounded bf16.  Pairs of elements go through packed fp32 arithmetic
-// (two values per instruction), which halves the instructions the rotation and
-// the norm issue; four 256-thread blocks stay resident per SM (64 registers, 32 KB
-// of ring each).  The kernel is
-// HBM-bound: two reads and two writes of n_tokens * n_heads * d bf16 values.
+// correctly rounded bf16.  The arithmetic runs in packed fp32 pairs (two values
+// per instruction), each pair holding the same position of two neighbouring
+// rotation pairs, so the cos/sin of those two pairs are packed alike and no
+// operand has to be duplicated or swapped per pass; four 256-thread blocks stay
+// resident per SM (64 registers, 32 KB of ring each).  The kernel is HBM-bound:
+// two reads and two writes of n_tokens * n_heads * d bf16 values.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -65,20 +66,13 @@ struct PrologueParams {
   RopeTables rope;
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&x)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-__device__ __forceinline__ uint4 f32x8_to_bf16(const float (&y)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = ptx::pack_bf16x2(y[2 * i], y[2 * i + 1]);
-  return make_uint4(w[0], w[1], w[2], w[3]);
+// 8 bf16 values (elements 0..7 = pairs 0..3) as two couples of pairs: a0[j] = the
+// first elements of pairs 2j, 2j+1; a1[j] = their second elements.
+__device__ __forceinline__ void bf16x8_to_couples(const uint4& u, float2 (&a0)[2], float2 (&a1)[2]) {
+  a0[0] = make_float2(__uint_as_float(u.x << 16), __uint_as_float(u.y << 16));
+  a1[0] = make_float2(__uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y & 0xFFFF0000u));
+  a0[1] = make_float2(__uint_as_float(u.z << 16), __uint_as_float(u.w << 16));
+  a1[1] = make_float2(__uint_as_float(u.z & 0xFFFF0000u), __uint_as_float(u.w & 0xFFFF0000u));
 }
 
 // 16-byte asynchronous global -> shared copy (bypasses the register file and L1).
@@ -128,12 +122,17 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const __g
     cp_async_commit();
   }
 
-  // gamma of this lane's 8 elements (fp32, exact)
-  float g[8];
+  // The lane's 8 elements as two couples of rotation pairs: couple j holds pairs
+  // 2j and 2j+1, a0 = (first elements of both pairs), a1 = (second elements), so
+  // one packed fp32 instruction works on the same position of two pairs and the
+  // pairs' cos/sin come packed the same way.
+  // gamma of this lane's 8 elements (fp32, exact), in couples
+  float2 g0[2], g1[2];
   const bool do_norm = gamma != nullptr;
   const bool any_norm = p.gamma_q != nullptr || p.gamma_k != nullptr;
   if (do_norm) {
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(gamma + chunk * 8), g);
+    const uint4 gw = *reinterpret_cast<const uint4*>(gamma + chunk * 8);
+    bf16x8_to_couples(gw, g0, g1);
   }
 
   int kind = 0;
@@ -153,7 +152,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const __g
   // |lo| <= ulp(hi)/2), from fp64: the rotation below then runs in fp32 with error-free
   // products.  The kRowsPerPass lanes that share a chunk need the same 4 pairs, so each
   // evaluates kPairsPerLane of them and the four values per pair are exchanged by shuffles.
-  float ch[4], cl[4], sh[4], sl[4];
+  float2 chi[2], clo[2], shi[2], slo[2];
   if (do_rope) {
     float mch[kPairsPerLane], mcl[kPairsPerLane], msh[kPairsPerLane], msl[kPairsPerLane];
 #pragma unroll
@@ -174,6 +173,7 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const __g
       msh[k] = static_cast<float>(sd);
       msl[k] = static_cast<float>(sd - static_cast<double>(msh[k]));
     }
+    float ch[4], cl[4], sh[4], sl[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int from = (k / kPairsPerLane) * kRowLanes + chunk;  // the lane that evaluated pair chunk*4+k
@@ -182,76 +182,94 @@ __global__ void __launch_bounds__(kPrologueThreads, 4) prologue_kernel(const __g
       sh[k] = __shfl_sync(0xffffffffu, msh[k % kPairsPerLane], from);
       sl[k] = __shfl_sync(0xffffffffu, msl[k % kPairsPerLane], from);
     }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      chi[j] = make_float2(ch[2 * j], ch[2 * j + 1]);
+      clo[j] = make_float2(cl[2 * j], cl[2 * j + 1]);
+      shi[j] = make_float2(sh[2 * j], sh[2 * j + 1]);
+      slo[j] = make_float2(sl[2 * j], sl[2 * j + 1]);
+    }
   }
 
   const float inv_d = 1.0f / static_cast<float>(D);
-  for (int pass = 0; pass < n_pass; ++pass) {
+  const int64_t in_step = static_cast<int64_t>(kHeadsPerPass) * p.in_head;
+  const int64_t out_step = static_cast<int64_t>(kHeadsPerPass) * p.out_head;
+  const uint16_t* refill = src + head_in_pass * p.in_head + kPrologueDepth * in_step;  // pass + kPrologueDepth
+  uint16_t* out = dst + head_in_pass * p.out_head;
+  int h = head_in_pass;
+  for (int pass = 0; pass < n_pass; ++pass, h += kHeadsPerPass, refill += in_step, out += out_step) {
     const int slot = pass % kPrologueDepth;
-    const int h = pass * kHeadsPerPass + head_in_pass;
     const bool live = h < n_heads;
     cp_async_wait<kPrologueDepth - 1>();  // this pass's group has landed
     uint4 raw = make_uint4(0, 0, 0, 0);
     if (live) raw = ring[warp][slot][lane];
 
-    float x[8];
-    bf16x8_to_f32(raw, x);
+    float2 a0[2], a1[2];
+    bf16x8_to_couples(raw, a0, a1);
     float r = 1.0f;
     if (any_norm) {  // warp-uniform: every lane joins the shuffles
-      float2 ss2 = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 xi = make_float2(x[2 * i], x[2 * i + 1]);
-        ss2 = __ffma2_rn(xi, xi, ss2);
-      }
+      float2 ss2 = __fmul2_rn(a0[0], a0[0]);
+      ss2 = __ffma2_rn(a1[0], a1[0], ss2);
+      ss2 = __ffma2_rn(a0[1], a0[1], ss2);
+      ss2 = __ffma2_rn(a1[1], a1[1], ss2);
       float ss = ss2.x + ss2.y;
 #pragma unroll
       for (int off = kRowLanes / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
       if (do_norm) {
         r = rsqrtf(fmaf(ss, inv_d, p.eps));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // exact
-          const float2 xg = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), make_float2(g[2 * i], g[2 * i + 1]));
-          x[2 * i] = xg.x;
-          x[2 * i + 1] = xg.y;
+        for (int j = 0; j < 2; ++j) {  // exact
+          a0[j] = __fmul2_rn(a0[j], g0[j]);
+          a1[j] = __fmul2_rn(a1[j], g1[j]);
         }
       }
     }
-    float y[8];
+    const float2 rr = make_float2(r, r);
+    float2 y0[2], y1[2];
     if (do_rope) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        // The pair a = (a0, a1) = x*gamma is exact in fp32.  As a complex product,
-        // y = a*c + ra*s with ra = (-a1, a0) and c, s each an unevaluated float pair
-        // (hi + lo).  The sine term's hi product is split into its rounded value q
-        // and exact error e (fma); m = a*c_hi + q then rounds once to within 2^-24
-        // of the result even where the two terms cancel, and the small terms
-        // (e, a*c_lo, ra*s_lo) carry the rest.  Each line works on both elements of
-        // the pair at once (packed fp32 pairs).
-        const float2 a = make_float2(x[2 * k], x[2 * k + 1]);
-        const float2 ra = make_float2(-x[2 * k + 1], x[2 * k]);
-        const float2 shi = make_float2(sh[k], sh[k]), slo = make_float2(sl[k], sl[k]);
-        const float2 chi = make_float2(ch[k], ch[k]), clo = make_float2(cl[k], cl[k]);
-        const float2 q = __fmul2_rn(ra, shi);
-        const float2 e = __ffma2_rn(ra, shi, make_float2(-q.x, -q.y));
-        const float2 m = __ffma2_rn(a, chi, q);
-        float2 lo = __ffma2_rn(a, clo, e);
-        lo = __ffma2_rn(ra, slo, lo);
-        const float2 yy = __fmul2_rn(__fadd2_rn(m, lo), make_float2(r, r));
-        y[2 * k] = yy.x;
-        y[2 * k + 1] = yy.y;
+      for (int j = 0; j < 2; ++j) {
+        // Each pair (a0, a1) = x*gamma is exact in fp32; its rotation is
+        //   y0 = a0*c - a1*s,  y1 = a1*c + a0*s,
+        // with c, s each an unevaluated float pair (hi + lo).  In each line the
+        // sine term's hi product is split into its rounded value q and exact error e
+        // (fma); m = (cosine term's hi product) + q then rounds once to within 2^-24
+        // of the result even where the two terms cancel, and the small terms (e and
+        // the lo products) carry the rest.
+        const float2 q0 = __fmul2_rn(a1[j], shi[j]);
+        const float2 nq0 = make_float2(-q0.x, -q0.y);
+        const float2 e0 = __ffma2_rn(a1[j], shi[j], nq0);          // a1*s_hi - q0, exact
+        const float2 m0 = __ffma2_rn(a0[j], chi[j], nq0);          // a0*c_hi - q0
+        float2 l0 = __ffma2_rn(a0[j], clo[j], make_float2(-e0.x, -e0.y));
+        l0 = __ffma2_rn(a1[j], make_float2(-slo[j].x, -slo[j].y), l0);
+        y0[j] = __fmul2_rn(__fadd2_rn(m0, l0), rr);
+        const float2 q1 = __fmul2_rn(a0[j], shi[j]);
+        const float2 e1 = __ffma2_rn(a0[j], shi[j], make_float2(-q1.x, -q1.y));  // a0*s_hi - q1, exact
+        const float2 m1 = __ffma2_rn(a1[j], chi[j], q1);           // a1*c_hi + q1
+        float2 l1 = __ffma2_rn(a1[j], clo[j], e1);
+        l1 = __ffma2_rn(a0[j], slo[j], l1);
+        y1[j] = __fmul2_rn(__fadd2_rn(m1, l1), rr);
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = x[i] * r;
+      for (int j = 0; j < 2; ++j) {
+        y0[j] = __fmul2_rn(a0[j], rr);
+        y1[j] = __fmul2_rn(a1[j], rr);
+      }
     }
     if (live && store_in_bounds(token < p.n_tokens && h < n_heads && chunk * 8 + 8 <= D)) {
-      *reinterpret_cast<uint4*>(dst + h * p.out_head) = f32x8_to_bf16(y);
+      // element 2i is the first of pair i: pair 2j + t sits in component t of couple j
+      uint4 o;
+      o.x = ptx::pack_bf16x2(y0[0].x, y1[0].x);
+      o.y = ptx::pack_bf16x2(y0[0].y, y1[0].y);
+      o.z = ptx::pack_bf16x2(y0[1].x, y1[1].x);
+      o.w = ptx::pack_bf16x2(y0[1].y, y1[1].y);
+      *reinterpret_cast<uint4*>(out) = o;
     }
     // Refill this slot (its value is consumed above) with the pass kPrologueDepth ahead; an
     // empty group keeps the group count in step at the tail.
-    const int nxt = pass + kPrologueDepth;
-    const int hn = nxt * kHeadsPerPass + head_in_pass;
-    if (nxt < n_pass && hn < n_heads) cp_async16(&ring[warp][slot][lane], src + hn * p.in_head);
+    if (pass + kPrologueDepth < n_pass && h + kPrologueDepth * kHeadsPerPass < n_heads)
+      cp_async16(&ring[warp][slot][lane], refill);
     cp_async_commit();
   }
 }
