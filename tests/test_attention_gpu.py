@@ -216,3 +216,37 @@ def test_ragged_bad_cu_seqlens_is_rejected_in_the_kernel(h3, orc, cu, max_seqlen
     got, got_lse = _gpu_varlen(h3, w.q, w.k, w.v, cu_ok)
     ro, rl = orc.attention(w.q, w.k, w.v, cu_ok)
     check_attention(bf16_bits_to_f64(got), ro, "valid launch after " + what, got_lse.T, rl, strict=True)
+
+
+def _ramped_case(lens, d, fac, seed):
+    """|Q| and |K| with key magnitudes growing along the sequence: every row's
+    maximum score grows from key tile to key tile (by ~8 log2 units per tile at
+    fac = 6, by more than 16 in 80% of tiles at fac = 16), so the running maximum
+    is raised and O rescaled in tensor memory many times per row."""
+    w = inputs.random_case(lens, 2, d, seed=seed)
+    q = np.abs(inputs.bf16_bits_to_f32(w.q))
+    k = np.abs(inputs.bf16_bits_to_f32(w.k))
+    pos = np.concatenate([np.arange(n) for n in lens]) if len(lens) else np.zeros(0)
+    span = np.concatenate([np.full(n, max(n, 1)) for n in lens]) if len(lens) else np.ones(0)
+    k = k * (1.0 + fac * pos / span).astype(np.float32)[:, None, None]
+    w.q = inputs.f32_to_bf16_bits(q)
+    w.k = inputs.f32_to_bf16_bits(k)
+    return w
+
+
+@pytest.mark.parametrize("fac,d", [(6.0, 128), (16.0, 128), (16.0, 64)])
+def test_running_max_grows_every_tile(h3, orc, fac, d):
+    # rows are peaked on the last keys (|o| up to ~3): the max bound is taken beyond
+    # the half-ulp storage cost, the plain mean bound holds
+    w = _ramped_case([1100], d, fac, seed=71)
+    o, lse = _gpu_dense(h3, w.q, w.k, w.v)
+    ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "ramped fac=%g d=%d" % (fac, d), lse.T, rl, strict=True,
+                    plain_max=False)
+
+
+def test_running_max_grows_every_tile_ragged(h3, orc):
+    w = _ramped_case([700, 1100, 0, 300], 128, 16.0, seed=72)
+    o, lse = _gpu_varlen(h3, w.q, w.k, w.v, w.cu_seqlens)
+    ro, rl = orc.attention(w.q, w.k, w.v, w.cu_seqlens)
+    check_attention(bf16_bits_to_f64(o), ro, "ramped ragged", lse.T, rl, strict=True, plain_max=False)
