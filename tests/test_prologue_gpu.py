@@ -173,3 +173,44 @@ def test_prologue_video_rows_sections(h3, orc, sections):
     rq, rk = _ref(orc, w)
     check_prologue(gq, rq, "sections %s q" % (sections,))
     check_prologue(gk, rk, "sections %s k" % (sections,))
+
+
+def _cancelling_rows(rng, pos, n, H, d, theta):
+    """bf16 rows whose rotation pairs nearly cancel: for pair i at angle
+    pos * theta^(-2i/d), x1 ~ x0 * cos/sin makes x0*cos - x1*sin vanish to the
+    rounding of x1, or x1 ~ -x0 * sin/cos does the same for x1*cos + x0*sin."""
+    i = np.arange(d // 2)
+    ang = pos[:, 0:1].astype(np.float64) * np.exp(-(2.0 * i / d) * np.log(theta))[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x0 = rng.uniform(0.5, 2.0, (n, H, d // 2)) * rng.choice([-1.0, 1.0], (n, H, d // 2))
+    x0 = inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(x0.astype(np.float32))).astype(np.float64)
+    with np.errstate(divide="ignore"):
+        ratio = np.where(rng.integers(0, 2, (n, H, d // 2)) == 0, (c / s)[:, None, :], (-s / c)[:, None, :])
+    usable = np.isfinite(ratio) & (np.abs(ratio) > 1.0 / 64) & (np.abs(ratio) < 64.0)
+    x1 = np.where(usable, x0 * np.where(usable, ratio, 0.0), rng.uniform(-2.0, 2.0, x0.shape))
+    x = np.empty((n, H, d))
+    x[..., 0::2] = x0
+    x[..., 1::2] = x1
+    return inputs.f32_to_bf16_bits(x.astype(np.float32))
+
+
+def test_prologue_rotation_cancellation(h3, orc):
+    # The two products of each rotated element nearly cancel, so the result is
+    # thousands of times smaller than its terms; a rotation with fp32 cos/sin and
+    # no error-free product misses the 1-ulp bound on ~0.1% of these elements (by up
+    # to thousands of ulps), the kernel's float-pair rotation must not.  Q without
+    # norm (no scale factor), K with a unit gamma (the RMS factor on top).
+    n, H, d = 2048, 4, 128
+    rng = np.random.default_rng(5)
+    w = inputs.make_workload("cancel", [n], H, d, seed=6, norm=True)
+    w.pos = np.zeros((n, 3), dtype=np.int32)
+    w.pos[:, 0] = rng.integers(0, 5000, n)
+    w.kind = np.full(n, 2, dtype=np.uint8)
+    w.q = _cancelling_rows(rng, w.pos, n, H, d, w.theta)
+    w.k = _cancelling_rows(rng, w.pos, n, H, d, w.theta)
+    w.gamma_q = None
+    w.gamma_k = inputs.f32_to_bf16_bits(np.ones(d, dtype=np.float32))
+    gq, gk = _run(h3, w)
+    rq, rk = _ref(orc, w)
+    check_prologue(gq, rq, "cancelling q")
+    check_prologue(gk, rk, "cancelling k")
