@@ -15,6 +15,8 @@ What pins what:
                   complex multiplication form; norm preservation; relative
                   position property; identities at position 0 / kind 0;
   norm + RoPE     one row recomputed step by step in 50-digit mpmath;
+  RoPE cancel     rows whose rotated elements nearly cancel, against 50-digit
+                  mpmath (fp64 value and bf16 rounding);
   attention       50-digit mpmath brute force (o and lse) on a ragged case;
                   torch scaled_dot_product_attention in float64; Q = 0 gives
                   the mean of V; one key gives V_0; constant V; permutation
@@ -275,6 +277,47 @@ def pin_norm_then_rope(orc):
         wb = np.array([nearest_bf16_bits(float(w)) for w in want], dtype=np.uint16)
         if not np.array_equal(y16[t, 0], wb):
             raise AssertionError("norm then rope: bf16 rounding of row %d differs" % t)
+
+
+def pin_rope_cancellation(orc):
+    """Rows whose rotated elements nearly cancel (x1 ~ x0 cos/sin, or x1 ~ -x0 sin/cos,
+    to the rounding of x1): the results are thousands of times smaller than their
+    terms; each is recomputed in 50-digit arithmetic and the oracle's bf16 rounding
+    must be the nearest bf16 of that value (and its fp64 value within a few double
+    ulps of the terms)."""
+    d = 128
+    rng = np.random.default_rng(11)
+    toks = [(2, (4097, 0, 0)), (2, (31233, 0, 0)), (1, (17, 40, 83)), (1, (3, 5, 7))]
+    n = len(toks)
+    pos = np.array([t[1] for t in toks], dtype=np.int32)
+    kind = np.array([t[0] for t in toks], dtype=np.uint8)
+    x = np.zeros((n, 1, d))
+    for t, (kd, p) in enumerate(toks):
+        for pair in range(d // 2):
+            a = _mp_angle(kd, p, pair)
+            c, s = float(mpmath.cos(a)), float(mpmath.sin(a))
+            x0 = float(bf16_value(to_bf16_bits_f32(np.array([rng.uniform(0.5, 2.0) * rng.choice([-1.0, 1.0])])))[0])
+            ratio = c / s if (pair % 2 == 0 and s != 0.0) else (-s / c if c != 0.0 else 0.0)
+            x1 = x0 * ratio if 1.0 / 64 < abs(ratio) < 64.0 else rng.uniform(-2.0, 2.0)
+            x[t, 0, 2 * pair], x[t, 0, 2 * pair + 1] = x0, x1
+    xb = to_bf16_bits_f32(x)
+    y, y16 = orc.rmsnorm_rope(xb, None, 0.0, pos, kind, SECTIONS, THETA)
+    xv = bf16_value(xb)
+    tiny = 0
+    for t, (kd, p) in enumerate(toks):
+        for pair in range(d // 2):
+            a = _mp_angle(kd, p, pair)
+            c, s = mpmath.cos(a), mpmath.sin(a)
+            x0, x1 = mpmath.mpf(float(xv[t, 0, 2 * pair])), mpmath.mpf(float(xv[t, 0, 2 * pair + 1]))
+            for j, w in ((2 * pair, x0 * c - x1 * s), (2 * pair + 1, x0 * s + x1 * c)):
+                scale = float(abs(x0) + abs(x1))
+                if abs(y[t, 0, j] - float(w)) > 4e-16 * scale * (1.0 + abs(float(a))):
+                    raise AssertionError("rope cancellation: token %d element %d: %r against %s" % (t, j, y[t, 0, j], w))
+                if int(y16[t, 0, j]) != nearest_bf16_bits(float(w)):
+                    raise AssertionError("rope cancellation: bf16 of token %d element %d differs" % (t, j))
+                tiny += abs(float(w)) < 1e-3 * scale
+    if tiny < n * d // 4:
+        raise AssertionError("rope cancellation: too few cancelling elements (%d)" % tiny)
 
 
 # ----------------------------------------------------------------------------------
@@ -601,6 +644,7 @@ ALL_PINS = [
     pin_rope_unit_vectors,
     pin_rope_properties,
     pin_norm_then_rope,
+    pin_rope_cancellation,
     pin_attention_brute_force,
     pin_attention_library,
     pin_attention_special_cases,
