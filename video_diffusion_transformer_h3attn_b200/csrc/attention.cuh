@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // ---- ragged descriptor check (before anything reads a sequence bound) -------------
   // cu_seqlens[0] = 0, non-decreasing, no sequence longer than max_seqlen (p.seqlen,
   // which sized the grid) and cu_seqlens[nseq] = total.  Every CTA reaches the same
-  // verdict; a descriptor that breaks a rule is reported in the sticky error bits
+  // decision; a descriptor that breaks a rule is reported in the sticky error bits
   // and the launch writes nothing.
   if (kVarlen) {
     bool bad = false;
